@@ -1,0 +1,439 @@
+/*
+ * ORACLE — test infrastructure only.
+ *
+ * A plain, slow, double-precision CPU statement of what the biased, routed
+ * attention call over MiniMax-H3's packed sequence computes.  Only the tests,
+ * the smoke check and the CPU-baseline leg of the benchmark may load it.  It
+ * shares no code, header or table with the CUDA library: it does not include
+ * the library's header and re-states every constant it needs.
+ *
+ * Sources (web pages; cited by title and section):
+ *  [FP]  "Flash Partitions for H3 native temporal alignment"
+ *        §1 "What receives the temporal bias?" (edge rule, penalty, score),
+ *        §3 "Decompose the same rule into positive contributions",
+ *        §4 "Why log-sum-exp is necessary" (partition merge).
+ *  [SLA] "H3 SLA Attention" node page, "How it works" (pooled matmul, top
+ *        1 - sparsity_ratio) and its inputs table (sparsity_ratio,
+ *        block_size, protect_audio).
+ *  [CFG] "Per-layer attention config LoRAs" (MiniMax-H3-Experiments
+ *        docs/attention.md), "Experimental: audio/text protection"
+ *        (sink_keys "prefix", sink_queries "audio"; 64-token query blocks).
+ *  [BRK] "H3 sparse-attention breakpoints: FL2VA, Ref2VA, and Turbo",
+ *        "Results at a glance" (what "10 %" of video KV means).
+ *  [WIKI] "TARA : alignement temporel natif pour les références MiniMax H3",
+ *        "La règle temporelle" (same rule and defaults).
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *  - logit scale 1/sqrt(d), natural-log softmax [FP §1];
+ *  - only output-video queries x guide-video keys are penalised [FP §1];
+ *  - dt = |t_q - t_k| from per-row times;
+ *  - pooled centroid = mean of the block's valid rows; pooled score =
+ *    Qp . Kp / sqrt(d); routing is per head;
+ *  - k = clamp(ceil((1 - s) * nV - 1e-9), 1, nV);
+ *  - ties in the pooled score go to the lower block index;
+ *  - a key block is forced (always attended) and a query block is dense iff
+ *    it overlaps any non-video row; every other block is a video block;
+ *  - dropped blocks leave the softmax (no pooled tail term);
+ *  - routing ignores the penalty; the exact penalty applies on the routed
+ *    output -> guide pairs.
+ *
+ * Segment ids: 0 text, 1 image-ref, 2 audio, 3 guide video, 4 output video.
+ * bf16 inputs are passed as their 16-bit patterns and widened exactly.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define SEG_GUIDE 3
+#define SEG_OUTPUT 4
+
+static inline int is_video(uint8_t s) { return s == SEG_GUIDE || s == SEG_OUTPUT; }
+
+static inline double bf16_to_f64(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+int oracle_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* [FP §1], [WIKI]: penalty(dt) = min(strength * (max(dt - window, 0) / falloff)^2, cap). */
+double oracle_penalty(double dt, double strength, double window, double falloff, double cap) {
+    double excess = dt - window;
+    if (excess < 0.0) excess = 0.0;
+    double r = excess / falloff;
+    double p = strength * r * r;
+    return p < cap ? p : cap;
+}
+
+/* [SLA] top (1 - sparsity_ratio) fraction of the video key blocks; [BRK] the
+ * fraction counts video KV tiles only.  Reading: round up, at least one. */
+int oracle_k(int n_video_blocks, double sparsity) {
+    double want = ceil((1.0 - sparsity) * (double)n_video_blocks - 1e-9);
+    int k = (int)want;
+    if (k < 1) k = 1;
+    if (k > n_video_blocks) k = n_video_blocks;
+    return k;
+}
+
+/* Block classes ([SLA] protect_audio: "blocks overlapping" text/cond/audio;
+ * [CFG] sink_keys "prefix", sink_queries "audio").  nonvideo[b] = 1 iff block
+ * b (rows [b*B, min(S,(b+1)*B))) holds a non-video row.  Returns the number of
+ * blocks ceil(S/B). */
+int oracle_block_classes(int S, int B, const uint8_t *seg, uint8_t *nonvideo) {
+    int nkb = (S + B - 1) / B;
+    for (int b = 0; b < nkb; ++b) {
+        int lo = b * B, hi = lo + B < S ? lo + B : S;
+        uint8_t nv = 0;
+        for (int r = lo; r < hi; ++r)
+            if (!is_video(seg[r])) nv = 1;
+        nonvideo[b] = nv;
+    }
+    return nkb;
+}
+
+/* Per-head mean of every block's valid rows ([SLA] "pooled centroids").
+ * x: bf16 [H][S][d]; out: [H][nKB][d]. */
+void oracle_pool(int H, int S, int d, int B, const uint16_t *x, double *out) {
+    int nkb = (S + B - 1) / B;
+#pragma omp parallel for schedule(static)
+    for (long hb = 0; hb < (long)H * nkb; ++hb) {
+        int h = (int)(hb / nkb), b = (int)(hb % nkb);
+        int lo = b * B, hi = lo + B < S ? lo + B : S;
+        double *o = out + (size_t)hb * d;
+        for (int c = 0; c < d; ++c) o[c] = 0.0;
+        for (int r = lo; r < hi; ++r) {
+            const uint16_t *row = x + ((size_t)h * S + r) * d;
+            for (int c = 0; c < d; ++c) o[c] += bf16_to_f64(row[c]);
+        }
+        for (int c = 0; c < d; ++c) o[c] /= (double)(hi - lo);
+    }
+}
+
+typedef struct {
+    double score;
+    int32_t block;
+} scored_block;
+
+/* score descending, then block index ascending */
+static int by_score_then_index(const void *a, const void *b) {
+    const scored_block *x = (const scored_block *)a, *y = (const scored_block *)b;
+    if (x->score > y->score) return -1;
+    if (x->score < y->score) return 1;
+    return (x->block > y->block) - (x->block < y->block);
+}
+
+static int ascending_i32(const void *a, const void *b) {
+    int32_t x = *(const int32_t *)a, y = *(const int32_t *)b;
+    return (x > y) - (x < y);
+}
+
+/*
+ * Block-sparse routing ([SLA] "How it works"): for every head and video query
+ * block i, score every video key block j with the pooled product
+ * Qp[i] . Kp[j] / sqrt(d), keep the k best (ties -> lower j), list them in
+ * ascending block order.
+ *
+ * sel: int32 [H][nV][k] (absolute block indices).  Optional outputs (NULL to
+ * skip): scores [H][nV][nV] (video q-block x video kv-block, both in
+ * ascending block order) and kth [H][nV] (the k-th best score).
+ * Returns k, or -1 if there is no video block.
+ */
+int oracle_route(int H, int S, int d, int B, double sparsity, const uint8_t *seg,
+                 const uint16_t *q, const uint16_t *k, int32_t *sel, double *scores,
+                 double *kth) {
+    int nkb = (S + B - 1) / B;
+    uint8_t *nonvideo = (uint8_t *)malloc((size_t)nkb);
+    oracle_block_classes(S, B, seg, nonvideo);
+    int nv = 0;
+    for (int b = 0; b < nkb; ++b) nv += !nonvideo[b];
+    if (nv == 0) {
+        free(nonvideo);
+        return -1;
+    }
+    int32_t *vid = (int32_t *)malloc(sizeof(int32_t) * (size_t)nv);
+    for (int b = 0, i = 0; b < nkb; ++b)
+        if (!nonvideo[b]) vid[i++] = b;
+    int kk = oracle_k(nv, sparsity);
+
+    double *qp = (double *)malloc(sizeof(double) * (size_t)H * nkb * d);
+    double *kp = (double *)malloc(sizeof(double) * (size_t)H * nkb * d);
+    oracle_pool(H, S, d, B, q, qp);
+    oracle_pool(H, S, d, B, k, kp);
+    double inv_sqrt_d = 1.0 / sqrt((double)d);
+
+#pragma omp parallel
+    {
+        scored_block *cand = (scored_block *)malloc(sizeof(scored_block) * (size_t)nv);
+#pragma omp for schedule(dynamic, 4)
+        for (long hi = 0; hi < (long)H * nv; ++hi) {
+            int h = (int)(hi / nv), i = (int)(hi % nv);
+            const double *a = qp + ((size_t)h * nkb + vid[i]) * d;
+            for (int j = 0; j < nv; ++j) {
+                const double *bvec = kp + ((size_t)h * nkb + vid[j]) * d;
+                double dot = 0.0;
+                for (int c = 0; c < d; ++c) dot += a[c] * bvec[c];
+                cand[j].score = dot * inv_sqrt_d;
+                cand[j].block = vid[j];
+                if (scores) scores[(size_t)hi * nv + j] = cand[j].score;
+            }
+            qsort(cand, (size_t)nv, sizeof(scored_block), by_score_then_index);
+            if (kth) kth[hi] = cand[kk - 1].score;
+            int32_t *dst = sel + (size_t)hi * kk;
+            for (int t = 0; t < kk; ++t) dst[t] = cand[t].block;
+            qsort(dst, (size_t)kk, sizeof(int32_t), ascending_i32);
+        }
+        free(cand);
+    }
+    free(qp);
+    free(kp);
+    free(vid);
+    free(nonvideo);
+    return kk;
+}
+
+/*
+ * The key blocks a query row attends.  Dense when sel is NULL or the row's
+ * block is non-video; otherwise the forced (non-video) blocks plus the routed
+ * list of the row's video query block.  Writes a 0/1 flag per block.
+ */
+static void attended_blocks(int nkb, const uint8_t *nonvideo, const int32_t *vid_index,
+                            const int32_t *sel, int kk, int H, int nv, int h, int qblock,
+                            uint8_t *use) {
+    if (sel == NULL || nonvideo[qblock]) {
+        for (int b = 0; b < nkb; ++b) use[b] = 1;
+        return;
+    }
+    for (int b = 0; b < nkb; ++b) use[b] = nonvideo[b];
+    const int32_t *lst = sel + ((size_t)h * nv + vid_index[qblock]) * kk;
+    for (int t = 0; t < kk; ++t) use[lst[t]] = 1;
+    (void)H;
+}
+
+/* score of one (query row, key row) pair, before any penalty: q.k / sqrt(d) */
+static inline double raw_score(const uint16_t *qr, const uint16_t *kr, int d, double inv_sqrt_d) {
+    double dot = 0.0;
+    for (int c = 0; c < d; ++c) dot += bf16_to_f64(qr[c]) * bf16_to_f64(kr[c]);
+    return dot * inv_sqrt_d;
+}
+
+/*
+ * Direct definition ([FP §1], [WIKI]).  For each requested (head, row):
+ *   x_j = q.k_j / sqrt(d) - p_j over the attended keys j,
+ *   p_j = penalty(|t_q - t_j|) if seg_q = output and seg_j = guide, else 0,
+ *   O = sum_j exp(x_j - m) v_j / sum_j exp(x_j - m),  LSE = m + ln sum_j exp(x_j - m).
+ * pen: {strength, window, falloff, cap} or NULL (no penalty).
+ * sel/kk: routed lists from a routing call, or NULL for dense attention.
+ * out_o: [n][d]; out_lse: [n].
+ */
+void oracle_attend(int H, int S, int d, int B, const uint8_t *seg, const float *times,
+                   const double *pen, const int32_t *sel, int kk, const uint16_t *q,
+                   const uint16_t *k, const uint16_t *v, int n, const int32_t *heads,
+                   const int32_t *rows, double *out_o, double *out_lse) {
+    int nkb = (S + B - 1) / B;
+    uint8_t *nonvideo = (uint8_t *)malloc((size_t)nkb);
+    oracle_block_classes(S, B, seg, nonvideo);
+    int32_t *vid_index = (int32_t *)malloc(sizeof(int32_t) * (size_t)nkb);
+    int nv = 0;
+    for (int b = 0; b < nkb; ++b) vid_index[b] = nonvideo[b] ? -1 : nv++;
+    double inv_sqrt_d = 1.0 / sqrt((double)d);
+
+#pragma omp parallel
+    {
+        double *x = (double *)malloc(sizeof(double) * (size_t)S);
+        uint8_t *use = (uint8_t *)malloc((size_t)nkb);
+#pragma omp for schedule(dynamic, 1)
+        for (int t = 0; t < n; ++t) {
+            int h = heads[t], i = rows[t];
+            attended_blocks(nkb, nonvideo, vid_index, sel, kk, H, nv, h, i / B, use);
+            const uint16_t *qr = q + ((size_t)h * S + i) * d;
+            int biased_row = pen != NULL && seg[i] == SEG_OUTPUT;
+            double m = -INFINITY;
+            for (int j = 0; j < S; ++j) {
+                if (!use[j / B]) continue;
+                double s = raw_score(qr, k + ((size_t)h * S + j) * d, d, inv_sqrt_d);
+                if (biased_row && seg[j] == SEG_GUIDE) {
+                    double dt = fabs((double)times[i] - (double)times[j]);
+                    s -= oracle_penalty(dt, pen[0], pen[1], pen[2], pen[3]);
+                }
+                x[j] = s;
+                if (s > m) m = s;
+            }
+            double l = 0.0;
+            double *o = out_o + (size_t)t * d;
+            for (int c = 0; c < d; ++c) o[c] = 0.0;
+            for (int j = 0; j < S; ++j) {
+                if (!use[j / B]) continue;
+                double w = exp(x[j] - m);
+                l += w;
+                const uint16_t *vr = v + ((size_t)h * S + j) * d;
+                for (int c = 0; c < d; ++c) o[c] += w * bf16_to_f64(vr[c]);
+            }
+            for (int c = 0; c < d; ++c) o[c] /= l;
+            out_lse[t] = m + log(l);
+        }
+        free(x);
+        free(use);
+    }
+    free(vid_index);
+    free(nonvideo);
+}
+
+/* ---- Flash-Partitions evaluation of the same rule ([FP §3], [FP §4]) ---- */
+
+typedef struct {
+    double time;
+    int32_t key;
+} timed_key;
+
+static int by_time(const void *a, const void *b) {
+    const timed_key *x = (const timed_key *)a, *y = (const timed_key *)b;
+    if (x->time < y->time) return -1;
+    if (x->time > y->time) return 1;
+    return (x->key > y->key) - (x->key < y->key);
+}
+
+/* Normalised softmax attention over one key partition: fills o[d] and returns
+ * its natural-log normaliser L = ln sum exp(x_j) over the partition (unbiased
+ * scores: the partition weight carries the penalty). */
+static double partition_attend(const uint16_t *qr, const uint16_t *kbase, const uint16_t *vbase,
+                               int d, double inv_sqrt_d, const int32_t *keys, int nkeys,
+                               double *x, double *o) {
+    double m = -INFINITY;
+    for (int t = 0; t < nkeys; ++t) {
+        x[t] = raw_score(qr, kbase + (size_t)keys[t] * d, d, inv_sqrt_d);
+        if (x[t] > m) m = x[t];
+    }
+    double l = 0.0;
+    for (int c = 0; c < d; ++c) o[c] = 0.0;
+    for (int t = 0; t < nkeys; ++t) {
+        double w = exp(x[t] - m);
+        l += w;
+        const uint16_t *vr = vbase + (size_t)keys[t] * d;
+        for (int c = 0; c < d; ++c) o[c] += w * bf16_to_f64(vr[c]);
+    }
+    for (int c = 0; c < d; ++c) o[c] /= l;
+    return m + log(l);
+}
+
+static inline double logaddexp(double a, double b) {
+    if (a == -INFINITY) return b;
+    if (b == -INFINITY) return a;
+    double hi = a > b ? a : b, lo = a > b ? b : a;
+    return hi + log1p(exp(lo - hi));
+}
+
+/*
+ * Same outputs as oracle_attend, reached by the partition algorithm: since
+ * 0 <= p <= cap, exp(-p) = exp(-cap) + [exp(-p) - exp(-cap)] with both terms
+ * non-negative ([FP §3]).  For a penalised (output-video) query the attended
+ * keys split into
+ *   N: non-guide keys, weight 1;
+ *   G: all guide keys, weight exp(-cap);
+ *   C_tau: guide keys with time tau where p(|t_q - tau|) < cap, weight
+ *          exp(-p) - exp(-cap) = exp(-cap) * expm1(cap - p);
+ * each partition is attended on its own (O_i, L_i) and the results merged by
+ * adjusted_L_i = L_i + log w_i, L = logsumexp_i adjusted_L_i,
+ * O = sum_i exp(adjusted_L_i - L) O_i ([FP §4]), with successive logaddexp.
+ * Any other query is one partition of weight 1.
+ */
+void oracle_attend_partitions(int H, int S, int d, int B, const uint8_t *seg,
+                              const float *times, const double *pen, const int32_t *sel,
+                              int kk, const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                              int n, const int32_t *heads, const int32_t *rows,
+                              double *out_o, double *out_lse) {
+    int nkb = (S + B - 1) / B;
+    uint8_t *nonvideo = (uint8_t *)malloc((size_t)nkb);
+    oracle_block_classes(S, B, seg, nonvideo);
+    int32_t *vid_index = (int32_t *)malloc(sizeof(int32_t) * (size_t)nkb);
+    int nv = 0;
+    for (int b = 0; b < nkb; ++b) vid_index[b] = nonvideo[b] ? -1 : nv++;
+    double inv_sqrt_d = 1.0 / sqrt((double)d);
+
+#pragma omp parallel
+    {
+        double *x = (double *)malloc(sizeof(double) * (size_t)S);
+        uint8_t *use = (uint8_t *)malloc((size_t)nkb);
+        int32_t *part = (int32_t *)malloc(sizeof(int32_t) * (size_t)S);
+        int32_t *plain = (int32_t *)malloc(sizeof(int32_t) * (size_t)S);
+        timed_key *guide = (timed_key *)malloc(sizeof(timed_key) * (size_t)S);
+        double *op = (double *)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 1)
+        for (int t = 0; t < n; ++t) {
+            int h = heads[t], i = rows[t];
+            attended_blocks(nkb, nonvideo, vid_index, sel, kk, H, nv, h, i / B, use);
+            const uint16_t *qr = q + ((size_t)h * S + i) * d;
+            const uint16_t *kb = k + (size_t)h * S * d;
+            const uint16_t *vb = v + (size_t)h * S * d;
+            double *o = out_o + (size_t)t * d;
+            int biased_row = pen != NULL && seg[i] == SEG_OUTPUT && pen[0] != 0.0 && pen[3] != 0.0;
+            int np = 0, ng = 0;
+            for (int j = 0; j < S; ++j) {
+                if (!use[j / B]) continue;
+                if (biased_row && seg[j] == SEG_GUIDE) {
+                    guide[ng].time = (double)times[j];
+                    guide[ng].key = j;
+                    ++ng;
+                } else {
+                    plain[np++] = j;
+                }
+            }
+            double L = -INFINITY;
+            for (int c = 0; c < d; ++c) o[c] = 0.0;
+            /* merge one normalised partition result (op, adjusted_L) into (o, L) */
+#define MERGE(adjL)                                                        \
+    do {                                                                   \
+        double newL = logaddexp(L, (adjL));                                \
+        double a = exp(L - newL), bw = exp((adjL) - newL);                 \
+        for (int c = 0; c < d; ++c) o[c] = a * o[c] + bw * op[c];          \
+        L = newL;                                                          \
+    } while (0)
+            if (np > 0) {
+                double Li = partition_attend(qr, kb, vb, d, inv_sqrt_d, plain, np, x, op);
+                MERGE(Li); /* weight 1: log 1 = 0 */
+            }
+            if (ng > 0) {
+                double cap = pen[3];
+                for (int g = 0; g < ng; ++g) part[g] = guide[g].key;
+                double Li = partition_attend(qr, kb, vb, d, inv_sqrt_d, part, ng, x, op);
+                MERGE(Li - cap); /* weight exp(-cap) */
+                qsort(guide, (size_t)ng, sizeof(timed_key), by_time);
+                for (int g0 = 0; g0 < ng;) {
+                    int g1 = g0;
+                    while (g1 < ng && guide[g1].time == guide[g0].time) ++g1;
+                    double dt = fabs((double)times[i] - guide[g0].time);
+                    double p = oracle_penalty(dt, pen[0], pen[1], pen[2], cap);
+                    if (p < cap) {
+                        /* w = exp(-p) - exp(-cap) = exp(-cap) * expm1(cap - p) > 0 */
+                        double logw = -cap + log(expm1(cap - p));
+                        for (int g = g0; g < g1; ++g) part[g - g0] = guide[g].key;
+                        double Lc = partition_attend(qr, kb, vb, d, inv_sqrt_d, part, g1 - g0, x, op);
+                        MERGE(Lc + logw);
+                    }
+                    g0 = g1;
+                }
+            }
+#undef MERGE
+            out_lse[t] = L;
+        }
+        free(x);
+        free(use);
+        free(part);
+        free(plain);
+        free(guide);
+        free(op);
+    }
+    free(vid_index);
+    free(nonvideo);
+}

@@ -1,0 +1,296 @@
+"""Pins of the fp64 oracle to values and identities fixed by the pages and by
+mathematics, independent of the oracle's own code.  CPU only."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import inputs
+import oracle
+from conftest import golden
+
+DEF = inputs.DEFAULT_PENALTY
+
+
+# ---------------------------------------------------------------- penalty --
+
+def test_penalty_worked_table():
+    """Flash Partitions page, section 3 table: penalty, factor, baseline, correction."""
+    for dt, pen, factor, baseline, corr in golden("penalty_table.txt"):
+        p = oracle.penalty(dt, *DEF)
+        assert abs(p - pen) <= 0.005 + 1e-12, (dt, p, pen)
+        assert abs(math.exp(-p) - factor) <= 5e-7
+        assert abs(math.exp(-DEF[3]) - baseline) <= 5e-7
+        assert abs((math.exp(-p) - math.exp(-DEF[3])) - corr) <= 5e-7 + 1e-12
+
+
+def test_penalty_saturation_threshold():
+    """Correction vanishes at window + falloff*sqrt(cap/strength) (~0.633 s); zero inside the window."""
+    (strength, window, falloff, cap, printed, decimals), = golden("saturation.txt")
+    thr = window + falloff * math.sqrt(cap / strength)
+    assert abs(thr - printed) <= 0.5 * 10 ** -int(decimals)
+    for dt in np.linspace(0.0, window, 11):
+        assert oracle.penalty(dt, strength, window, falloff, cap) == 0.0
+    for dt in [thr + 1e-9, thr + 0.01, 0.8, 1.5, 10.0]:
+        p = oracle.penalty(dt, strength, window, falloff, cap)
+        assert p == cap and math.exp(-p) - math.exp(-cap) == 0.0
+    for dt in [window + 1e-6, 0.3, 0.5, thr - 1e-6]:
+        p = oracle.penalty(dt, strength, window, falloff, cap)
+        assert 0.0 < p < cap and math.exp(-p) - math.exp(-cap) > 0.0
+
+
+def test_penalty_monotone_bounded_and_reductions():
+    dts = np.linspace(0, 3, 3001)
+    ps = [oracle.penalty(t, *DEF) for t in dts]
+    assert all(0.0 <= p <= DEF[3] for p in ps)
+    assert all(b >= a for a, b in zip(ps, ps[1:]))
+    # strength = 0 or cap = 0 removes the penalty (Flash Partitions page, section 4 end)
+    assert all(oracle.penalty(t, 0.0, 0.2, 0.25, 6.0) == 0.0 for t in dts)
+    assert all(oracle.penalty(t, 2.0, 0.2, 0.25, 0.0) == 0.0 for t in dts)
+
+
+def test_decomposition_identity():
+    """exp(-p) = exp(-cap) + [exp(-p) - exp(-cap)], both terms >= 0 (section 3)."""
+    cap = DEF[3]
+    for t in np.linspace(0, 2, 401):
+        p = oracle.penalty(t, *DEF)
+        base, corr = math.exp(-cap), math.exp(-p) - math.exp(-cap)
+        assert base > 0 and corr >= 0
+        assert abs(base + corr - math.exp(-p)) <= 1e-15
+
+
+# ------------------------------------------------------------- helpers --
+
+def _tiny(seed=7, frames=6, gtok=20, otok=22, text=20, audio=30, H=2, d=32, cluster=0.0):
+    segs = [inputs.Segment(inputs.SEG_TEXT, text), inputs.Segment(inputs.SEG_AUDIO, audio),
+            inputs.Segment(inputs.SEG_GUIDE, frames * gtok, frames),
+            inputs.Segment(inputs.SEG_OUTPUT, frames * otok, frames)]
+    cfg = inputs.custom(H, d, segs, seed, cluster_norm=cluster, penalty=DEF)
+    seg, times, _ = cfg.layout()
+    q = inputs.tensor(cfg, inputs.TENSOR_Q)
+    k = inputs.tensor(cfg, inputs.TENSOR_K)
+    v = inputs.tensor(cfg, inputs.TENSOR_V)
+    return cfg, seg, times, q, k, v
+
+
+def _f64(x):
+    return torch.from_numpy(inputs.bf16_bits_to_f64(x))
+
+
+def _sdpa(q, k, v, mask=None):
+    """torch's scaled_dot_product_attention in fp64 on CPU (library routine)."""
+    return torch.nn.functional.scaled_dot_product_attention(
+        _f64(q)[None], _f64(k)[None], _f64(v)[None], attn_mask=mask).numpy()[0]
+
+
+def _bias(seg, times, pen):
+    """-penalty on output-query x guide-key pairs (edge rule of the Flash Partitions page, section 1)."""
+    S = len(seg)
+    b = np.zeros((S, S))
+    qi = np.where(seg == inputs.SEG_OUTPUT)[0]
+    kj = np.where(seg == inputs.SEG_GUIDE)[0]
+    for i in qi:
+        for j in kj:
+            b[i, j] = -oracle.penalty(abs(float(times[i]) - float(times[j])), *pen)
+    return torch.from_numpy(b)
+
+
+# ------------------------------------------------------------ attention --
+
+@pytest.mark.parametrize("pen", [None, (0.0, 0.2, 0.25, 6.0), (2.0, 0.2, 0.25, 0.0)])
+def test_unbiased_reduces_to_library_softmax(pen):
+    """No penalty, strength 0 or cap 0 -> textbook softmax(QK^T/sqrt(d))V (torch SDPA, fp64)."""
+    cfg, seg, times, q, k, v = _tiny()
+    o, lse = oracle.attend(q, k, v, seg, times, pen=pen)
+    ref = _sdpa(q, k, v)
+    H, S, d = q.shape
+    assert np.abs(o.reshape(H, S, d) - ref).max() < 1e-12
+    s = torch.einsum("hid,hjd->hij", _f64(q), _f64(k)) / math.sqrt(d)
+    assert np.abs(lse.reshape(H, S) - torch.logsumexp(s, -1).numpy()).max() < 1e-12
+
+
+@pytest.mark.parametrize("pen", [DEF, (0.5, 0.1, 0.3, 3.0), (8.0, 0.2, 0.25, 12.0)])
+def test_biased_matches_library_with_explicit_bias(pen):
+    """Penalty on output->guide edges only == SDPA with the explicit additive bias."""
+    cfg, seg, times, q, k, v = _tiny()
+    o, lse = oracle.attend(q, k, v, seg, times, pen=pen)
+    bias = _bias(seg, times, pen)
+    ref = _sdpa(q, k, v, mask=bias)
+    H, S, d = q.shape
+    assert np.abs(o.reshape(H, S, d) - ref).max() < 1e-12
+    s = torch.einsum("hid,hjd->hij", _f64(q), _f64(k)) / math.sqrt(d) + bias
+    assert np.abs(lse.reshape(H, S) - torch.logsumexp(s, -1).numpy()).max() < 1e-12
+
+
+def test_bias_changes_only_output_rows():
+    cfg, seg, times, q, k, v = _tiny()
+    o0, _ = oracle.attend(q, k, v, seg, times, pen=None)
+    o1, _ = oracle.attend(q, k, v, seg, times, pen=DEF)
+    H, S, d = q.shape
+    diff = np.abs(o1 - o0).reshape(H, S, d).max(axis=(0, 2))
+    assert np.all(diff[seg != inputs.SEG_OUTPUT] == 0.0)
+    assert np.all(diff[seg == inputs.SEG_OUTPUT] > 0.0)
+
+
+@pytest.mark.parametrize("pen", [DEF, (0.5, 0.1, 0.3, 3.0), (8.0, 0.2, 0.25, 12.0),
+                                 (2.0, 0.0, 0.25, 1.0), (2.0, 0.2, 0.05, 6.0)])
+@pytest.mark.parametrize("layout", [dict(), dict(frames=9, gtok=13, otok=11),
+                                    dict(frames=4, gtok=33, otok=31, text=7, audio=5)])
+def test_partition_merge_equals_direct(pen, layout):
+    """Flash-Partitions decomposition + log-sum-exp merge (sections 3-4) equals the direct
+    rule at several strengths/caps and frame layouts (frames straddle 16-row blocks)."""
+    cfg, seg, times, q, k, v = _tiny(**layout)
+    o1, l1 = oracle.attend(q, k, v, seg, times, pen=pen, B=16)
+    o2, l2 = oracle.attend_partitions(q, k, v, seg, times, pen=pen, B=16)
+    assert np.abs(o1 - o2).max() < 1e-12
+    assert np.abs(l1 - l2).max() < 1e-12
+
+
+def test_output_is_convex_combination():
+    cfg, seg, times, q, k, v = _tiny()
+    o, _ = oracle.attend(q, k, v, seg, times, pen=DEF)
+    H, S, d = q.shape
+    vf = inputs.bf16_bits_to_f64(v)
+    o = o.reshape(H, S, d)
+    assert np.all(o <= vf.max(axis=1, keepdims=True) + 1e-12)
+    assert np.all(o >= vf.min(axis=1, keepdims=True) - 1e-12)
+
+
+# -------------------------------------------------------------- routing --
+
+def _route_case(seed=11, H=3, d=32, frames=8, tok=48):
+    segs = [inputs.Segment(inputs.SEG_TEXT, 40), inputs.Segment(inputs.SEG_AUDIO, 50),
+            inputs.Segment(inputs.SEG_OUTPUT, frames * tok, frames)]
+    cfg = inputs.custom(H, d, segs, seed, cluster_norm=2.0)
+    seg, times, _ = cfg.layout()
+    return cfg, seg, times, inputs.tensor(cfg, 0), inputs.tensor(cfg, 1), inputs.tensor(cfg, 2)
+
+
+def test_pool_is_block_mean():
+    cfg, seg, times, q, k, v = _route_case()
+    B = 16
+    p = oracle.pool(q, B)
+    x = inputs.bf16_bits_to_f64(q)
+    H, S, d = x.shape
+    for b in range(p.shape[1]):
+        ref = x[:, b * B:min(S, (b + 1) * B)].mean(axis=1)
+        assert np.abs(p[:, b] - ref).max() < 1e-14
+
+
+def test_block_classes_and_k():
+    seg = np.array([0] * 70 + [2] * 10 + [3] * 100 + [4] * 50, np.uint8)  # S = 230
+    cls = oracle.block_classes(seg, 64)
+    assert list(cls) == [1, 1, 0, 0]          # block 1 mixes audio rows 64..79 and video
+    for nv in [1, 2, 7, 246, 741, 1794]:
+        for s in [0.0, 0.6, 0.85, 0.9, 0.999]:
+            kk = oracle.k_for(nv, s)
+            assert 1 <= kk <= nv
+            assert kk >= (1 - s) * nv - 1e-6 and (kk - 1 < (1 - s) * nv or kk == 1)
+    assert oracle.k_for(1794, 0.90) == 180 and oracle.k_for(246, 0.85) == 37
+    assert oracle.k_for(50, 0.0) == 50
+
+
+@pytest.mark.parametrize("sparsity", [0.5, 0.75, 0.9])
+def test_route_matches_library_topk(sparsity):
+    """Pooled scores by torch (mean + matmul) and selection by torch.topk give the same sets."""
+    cfg, seg, times, q, k, v = _route_case()
+    B = 16
+    sel, scores, kth = oracle.route(q, k, seg, sparsity, B=B, want_scores=True)
+    cls = oracle.block_classes(seg, B)
+    vid = np.where(cls == 0)[0]
+    H, S, d = q.shape
+    nkb = (S + B - 1) // B
+
+    def pooled(x):
+        x = _f64(x)
+        return torch.stack([x[:, b * B:min(S, (b + 1) * B)].mean(1) for b in range(nkb)], 1)
+    qp, kp = pooled(q)[:, vid], pooled(k)[:, vid]
+    ref = torch.einsum("hid,hjd->hij", qp, kp) / math.sqrt(d)
+    assert np.abs(scores - ref.numpy()).max() < 1e-12
+    kk = sel.shape[-1]
+    top = torch.topk(ref, kk, dim=-1).indices.numpy()
+    for h in range(H):
+        for i in range(len(vid)):
+            assert sorted(vid[top[h, i]].tolist()) == sel[h, i].tolist()
+            assert kth[h, i] == pytest.approx(float(torch.sort(ref[h, i], descending=True).values[kk - 1]), abs=1e-15)
+
+
+def test_route_invariants_and_dense_limit():
+    cfg, seg, times, q, k, v = _route_case()
+    B = 16
+    cls = oracle.block_classes(seg, B)
+    vid = set(np.where(cls == 0)[0].tolist())
+    sel, _, _ = oracle.route(q, k, seg, 0.8, B=B)
+    for lst in sel.reshape(-1, sel.shape[-1]):
+        assert list(lst) == sorted(set(lst.tolist())) and set(lst.tolist()) <= vid
+    sel0, _, _ = oracle.route(q, k, seg, 0.0, B=B)
+    assert np.all(sel0 == np.array(sorted(vid))[None, None, :])
+
+
+def test_route_tie_goes_to_lower_block():
+    """Two identical key blocks score exactly alike: the lower index must win."""
+    cfg, seg, times, q, k, v = _route_case(H=1)
+    B = 16
+    cls = oracle.block_classes(seg, B)
+    vid = np.where(cls == 0)[0]
+    k = k.copy()
+    a, b = int(vid[3]), int(vid[9])
+    k[:, b * B:(b + 1) * B] = k[:, a * B:(a + 1) * B]
+    nv = len(vid)
+    sel, scores, kth = oracle.route(q, k, seg, 0.0, B=B, want_scores=True)
+    for s in np.linspace(0.05, 0.95, 19):
+        sel, scores, kth = oracle.route(q, k, seg, s, B=B, want_scores=True)
+        for i in range(nv):
+            row = sel[0, i].tolist()
+            if (a in row) != (b in row):        # cut falls between the twins
+                assert a in row and b not in row
+
+
+def test_routed_attention_matches_masked_library_softmax():
+    """Routed attention == SDPA with -inf on the key blocks a query block does not attend."""
+    cfg, seg, times, q, k, v = _route_case(H=2, d=32, frames=6, tok=40)
+    B = 16
+    sel, _, _ = oracle.route(q, k, seg, 0.7, B=B)
+    o, lse = oracle.attend(q, k, v, seg, times, pen=None, sel=sel, B=B)
+    cls = oracle.block_classes(seg, B)
+    vid_index = {b: i for i, b in enumerate(np.where(cls == 0)[0])}
+    H, S, d = q.shape
+    nkb = (S + B - 1) // B
+    ref = np.empty((H, S, d))
+    for h in range(H):
+        mask = torch.zeros(S, S, dtype=torch.float64)
+        for i in range(S):
+            qb = i // B
+            if cls[qb]:
+                continue
+            allowed = set(np.where(cls == 1)[0].tolist()) | set(sel[h, vid_index[qb]].tolist())
+            for kb in range(nkb):
+                if kb not in allowed:
+                    mask[i, kb * B:(kb + 1) * B] = -math.inf
+        ref[h] = torch.nn.functional.scaled_dot_product_attention(
+            _f64(q)[h:h + 1], _f64(k)[h:h + 1], _f64(v)[h:h + 1], attn_mask=mask).numpy()[0]
+    assert np.abs(o.reshape(H, S, d) - ref).max() < 1e-12
+    # the partition path agrees on routed lists too
+    o2, l2 = oracle.attend_partitions(q, k, v, seg, times, pen=DEF, sel=sel, B=B)
+    o3, l3 = oracle.attend(q, k, v, seg, times, pen=DEF, sel=sel, B=B)
+    assert np.abs(o2 - o3).max() < 1e-12 and np.abs(l2 - l3).max() < 1e-12
+
+
+def test_sparsity_zero_equals_dense():
+    cfg, seg, times, q, k, v = _route_case(H=2, frames=5, tok=40)
+    B = 16
+    sel, _, _ = oracle.route(q, k, seg, 0.0, B=B)
+    o1, l1 = oracle.attend(q, k, v, seg, times, pen=DEF, sel=sel, B=B)
+    o2, l2 = oracle.attend(q, k, v, seg, times, pen=DEF, sel=None, B=B)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_sampled_rows_equal_full_rows():
+    cfg, seg, times, q, k, v = _tiny()
+    H, S, d = q.shape
+    o, lse = oracle.attend(q, k, v, seg, times, pen=DEF)
+    heads = np.array([0, 1, 1, 0]); rows = np.array([0, S - 1, 100, 250])
+    o2, l2 = oracle.attend(q, k, v, seg, times, pen=DEF, heads=heads, rows=rows)
+    assert np.array_equal(o2, o.reshape(H, S, d)[heads, rows])
+    assert np.array_equal(l2, lse.reshape(H, S)[heads, rows])
