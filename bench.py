@@ -1,0 +1,400 @@
+"""Benchmark of one call of the hot path: block routing (pool + pooled score +
+top-k) followed by the fused biased attention over the routed tiles, at the
+full H3 packing S = 116,883, H = 56, d = 128, sparsity 0.90, default temporal
+penalty (workload "full combined").
+
+Prints one JSON line.  value = effective attention TFLOP/s over all ranks
+(4*d FLOPs per attended (query, key, head) triple, valid pairs only) with the
+inputs resident in HBM; e2e = the same metric through the C ABI with host
+buffers (host->device copy of Q, K, V, seg, times and device->host copy of O
+inside the timed region).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU: torchrun, one process per GPU; every rank runs its own independent
+call (its own seeded input), no collective on the data path (weak scaling).
+The reference arm times the fp64 CPU oracle on a bounded sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import inputs  # noqa: E402
+
+CONFIG_ID = 5
+WORKLOAD = "full combined: S=116883 (text 256|image-ref 1013|audio 810|guide 27x2126|output 27x2126), " \
+           "H=56, d=128, bf16, block 64, sparsity 0.90 (k=180 of 1794 video KV blocks), default penalty"
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def effective_pairs(p, sel: np.ndarray | None) -> int:
+    """Sum over heads and query rows of the attended (valid) keys."""
+    S, B = p.S, 64
+    nkb = p.n_blocks
+    rows = np.minimum(B, S - np.arange(nkb) * B).astype(np.int64)
+    if sel is None:
+        return int(p.H) * S * S
+    forced_keys = int(rows[:p.first_video_block].sum())
+    dense_pairs = int(rows[:p.first_video_block].sum()) * S
+    routed_keys = rows[sel].sum(axis=-1) + forced_keys      # [H][nV]
+    vrows = rows[p.first_video_block:]
+    return int(p.H) * dense_pairs + int((routed_keys * vrows[None, :]).sum())
+
+
+def executed_mma_pairs(p, sel: np.ndarray | None) -> int:
+    """(query, key) pairs the tensor cores actually process: per 128-row tile, the union
+    of its two query blocks' key lists, rounded up to 128-key tiles."""
+    nkb = p.n_blocks
+    n_tiles_q = (nkb + 1) // 2
+    if sel is None:
+        return int(p.H) * n_tiles_q * 128 * ((nkb + 1) // 2) * 128
+    total = 0
+    fvb = p.first_video_block
+    for t in range(n_tiles_q):
+        a, b = 2 * t, 2 * t + 1
+        if a < fvb or (b < nkb and b < fvb):
+            total += p.H * ((nkb + 1) // 2)
+            continue
+        la = sel[:, a - fvb]
+        if b < nkb:
+            lb = sel[:, b - fvb]
+            for h in range(p.H):
+                u = np.union1d(la[h], lb[h]).size + fvb
+                total += (u + 1) // 2
+        else:
+            total += p.H * ((la.shape[1] + fvb + 1) // 2)
+    return int(total) * 128 * 128
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        with open(self.file.name) as f:
+            lines = [ln.strip() for ln in f if ln.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def oracle_sample(cfg, q, k, v, seg, times, pen, sparsity, budget_s: float, head: int = 0):
+    """Time the fp64 oracle on a bounded sample of the workload: full routing of one
+    head plus attention for sampled query rows of that head (dense and routed rows).
+    Returns (effective FLOPs done, seconds, description)."""
+    import oracle
+
+    t0 = time.perf_counter()
+    qh, kh, vh = q[head:head + 1], k[head:head + 1], v[head:head + 1]
+    sel, _, _ = oracle.route(qh, kh, seg, sparsity)
+    t_route = time.perf_counter() - t0
+    nkb = (cfg.S + 63) // 64
+    cls = oracle.block_classes(seg)
+    fvb = int(cls.sum())
+    rng = np.random.default_rng(1234)
+    blocks = [0, fvb - 1, fvb, nkb - 1] + list(rng.integers(fvb, nkb, size=64))
+    rows_done, flops = 0, 0
+    rows_all = []
+    for b in blocks:
+        for r in (0, 21, 42, 63):
+            x = int(b) * 64 + r
+            if x < cfg.S:
+                rows_all.append(x)
+    rows_per_key = np.minimum(64, cfg.S - np.arange(nkb) * 64)
+    forced_keys = int(rows_per_key[:fvb].sum())
+    i = 0
+    while i < len(rows_all) and time.perf_counter() - t0 < budget_s:
+        chunk = np.array(rows_all[i:i + 8], np.int32)
+        oracle.attend(qh, kh, vh, seg, times, pen=pen, sel=sel, heads=np.zeros(len(chunk), np.int32), rows=chunk)
+        for x in chunk:
+            qb = x // 64
+            keys = cfg.S if qb < fvb else forced_keys + int(rows_per_key[sel[0, qb - fvb]].sum())
+            flops += 4 * cfg.d * keys
+        rows_done += len(chunk)
+        i += 8
+    secs = time.perf_counter() - t0
+    desc = (f"oracle fp64 on {oracle.threads()} threads: routing of head {head} "
+            f"({t_route:.2f} s, {int(cls.size - fvb)}^2 pooled scores) + attention of {rows_done} sampled "
+            f"query rows of that head (dense prefix rows and routed video rows)")
+    return flops, secs, desc, rows_done
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the fp64 CPU oracle, rank 0 only."""
+    if rank != 0:
+        return
+    cfg = inputs.CONFIGS[CONFIG_ID]
+    seg, times, _ = cfg.layout()
+    small = inputs.custom(1, cfg.d, cfg.segments, cfg.seed, cluster_norm=cfg.cluster_norm)
+    q, k, v = (inputs.tensor(small, t) for t in range(3))
+    import oracle
+
+    total_flops, total_s, desc = 0, 0.0, ""
+    for i in range(args.warmup + args.steps):
+        f, s, desc, _ = oracle_sample(cfg, q, k, v, seg, times, cfg.penalty, cfg.sparsities[0], budget_s=4.0)
+        if i >= args.warmup:
+            total_flops += f
+            total_s += s
+    value = total_flops / total_s / 1e12
+    line = {"metric": "effective attention TFLOP/s (S=116883, H=56, d=128, sparsity 0.90, penalty on)",
+            "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator)", "impl": "reference",
+            "config": {"workload": WORKLOAD, "sample": "per step: bounded oracle sample of the workload"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.threads(), "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import biased_attention_video_b200 as h3
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = inputs.CONFIGS[CONFIG_ID]
+    seed = cfg.seed + rank
+    seg, times, _ = cfg.layout()
+    H, S, d = cfg.H, cfg.S, cfg.d
+    sparsity = cfg.sparsities[0]
+    pen = cfg.penalty
+
+    # inputs generated straight into pinned host memory (also the e2e sources)
+    n = H * S * d
+    host = {t: torch.empty(n, dtype=torch.int16, pin_memory=True) for t in ("q", "k", "v")}
+    for i, t in enumerate(("q", "k", "v")):
+        inputs.tensor(cfg, i, out=host[t].numpy().view(np.uint16), seed=seed)
+    seg_h = torch.from_numpy(seg).pin_memory()
+    times_h = torch.from_numpy(times).pin_memory()
+    o_h = torch.empty(n, dtype=torch.int16, pin_memory=True)
+    qd, kd, vd = (host[t].to(dev).view(torch.bfloat16).view(H, S, d) for t in ("q", "k", "v"))
+    seg_d, times_d = seg_h.to(dev), times_h.to(dev)
+    p = h3.plan(H, S, d, seg, sparsity=sparsity)
+    ws = h3.workspace(p, dev)
+    sel = torch.empty((H, p.n_video_blocks, p.k), dtype=torch.int32, device=dev)
+    o = torch.empty_like(qd)
+    stream = torch.cuda.current_stream(dev)
+
+    ev = {"r0": [], "r1": [], "f0": [], "f1": []}
+
+    def step(record=False):
+        if record:
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            e[0].record(stream)
+        h3.route(p, qd, kd, ws, kv_sel=sel)
+        if record:
+            e[1].record(stream)
+            e[2].record(stream)
+        h3.forward(p, qd, kd, vd, seg_d, times_d, pen=pen, kv_sel=sel, ws=ws, out=o)
+        if record:
+            e[3].record(stream)
+            for key, x in zip(("r0", "r1", "f0", "f1"), e):
+                ev[key].append(x)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    status = h3.check(ws)
+    if status != h3.OK:
+        raise RuntimeError(f"device status {status} after warm-up")
+    sel_h = sel.cpu().numpy()
+    pairs = effective_pairs(p, sel_h)
+    eff_flops = 4 * d * pairs
+    mma_pairs = executed_mma_pairs(p, sel_h)
+
+    if world > 1:
+        dist.barrier()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for _ in range(args.steps):
+        step(record=True)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    status = h3.check(ws)
+    if status != h3.OK:
+        raise RuntimeError(f"device status {status} in timed region")
+    ms = t_start.elapsed_time(t_end)
+    route_ms = sum(a.elapsed_time(b) for a, b in zip(ev["r0"], ev["r1"])) / args.steps
+    fwd_ms = sum(a.elapsed_time(b) for a, b in zip(ev["f0"], ev["f1"])) / args.steps
+
+    # end to end through the C ABI from pinned host buffers
+    h2d = 3 * n * 2 + S + 4 * S
+    d2h = n * 2
+    qh_v, kh_v, vh_v = host["q"], host["k"], host["v"]
+
+    def e2e_step():
+        qd.view(torch.int16).view(-1).copy_(qh_v, non_blocking=True)
+        kd.view(torch.int16).view(-1).copy_(kh_v, non_blocking=True)
+        vd.view(torch.int16).view(-1).copy_(vh_v, non_blocking=True)
+        seg_d.copy_(seg_h, non_blocking=True)
+        times_d.copy_(times_h, non_blocking=True)
+        h3.route(p, qd, kd, ws, kv_sel=sel)
+        h3.forward(p, qd, kd, vd, seg_d, times_d, pen=pen, kv_sel=sel, ws=ws, out=o)
+        o_h.copy_(o.view(torch.int16).view(-1), non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if h3.check(ws) != h3.OK:
+        raise RuntimeError("device status after e2e")
+
+    # max over ranks
+    t = torch.tensor([ms, e2e_ms, fwd_ms, route_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms, e2e_ms, fwd_ms, route_ms = (float(x) for x in t.cpu())
+
+    if rank != 0:
+        return
+    peaks, peak_kind = measured_peaks()
+    ms_step = ms / args.steps
+    value = world * eff_flops * args.steps / (ms * 1e-3) / 1e12
+    e2e_value = world * eff_flops * args.steps / (e2e_ms * 1e-3) / 1e12
+    attn_tflops = eff_flops / (fwd_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    route_bytes = 2 * H * p.n_video_blocks * 64 * d * 2  # Q and K video rows, read once by the pool
+    line = {
+        "metric": "effective attention TFLOP/s (S=116883, H=56, d=128, sparsity 0.90, penalty on)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded counter-based generator, cluster-mean Q/K)",
+        "config": {"workload": WORKLOAD, "H": H, "S": S, "d": d, "block": 64, "sparsity": sparsity,
+                   "k": int(p.k), "seed": seed, "l2": "no flush: Q+K+V = 5.0 GB per step, far above the 126 MB L2",
+                   "effective_tflop_per_call": eff_flops / 1e12,
+                   "executed_mma_tflop_per_call": 4 * d * mma_pairs / 1e12,
+                   "route_ms": route_ms, "attention_ms": fwd_ms},
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": attn_tflops / peak, "traffic": None,
+                     "kernel": "attn_kernel (fused routed attention); achieved = effective FLOPs per launch / "
+                               "CUDA-event time of the forward call (kv_desc prep + attention)",
+                     "peak_source": f"{peak_kind} bf16_tflops_sustained"},
+        "routing": {"ms": route_ms, "bytes_read": route_bytes, "gbs": route_bytes / (route_ms * 1e-3) / 1e9,
+                    "hbm_peak_gbs": peaks["hbm_gbs"]},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms / args.steps},
+    }
+    if not args.no_cpu_baseline and world == 1:
+        small = inputs.custom(1, d, cfg.segments, seed, cluster_norm=cfg.cluster_norm)
+        qs, ks, vs = (inputs.tensor(small, i) for i in range(3))
+        f, s, desc, _ = oracle_sample(cfg, qs, ks, vs, seg, times, pen, sparsity, budget_s=args.cpu_budget)
+        import oracle
+        line["cpu_baseline"] = {"value": f / s / 1e12, "unit": "TFLOP/s", "cores": oracle.threads(),
+                                "kind": "oracle", "sample": desc}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

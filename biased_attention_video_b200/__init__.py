@@ -1,0 +1,204 @@
+"""Python binding of libh3attn (biased, block-routed attention over MiniMax-H3's
+packed sequence on B200).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  PyTorch supplies device memory and the current stream.  There is no
+fallback: if libh3attn.so cannot be loaded, every call raises.
+
+Tensors: q, k, v, o bf16 [H, S, d] contiguous CUDA; seg uint8 [S]; times
+float32 [S]; kv_sel int32 [H, n_video_blocks, k].
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+import torch
+
+from . import build as _build
+
+OK, EINVAL, EUNSUPPORTED, EALIGN, ECUDA, ETIMEOUT, EWORKSPACE, EDATA = 0, -1, -2, -3, -4, -5, -6, -7
+SEG_TEXT, SEG_IMAGE_REF, SEG_AUDIO, SEG_GUIDE, SEG_OUTPUT = 0, 1, 2, 3, 4
+
+# every symbol the C header declares
+EXPORTS = ("h3attn_plan_init", "h3attn_workspace_bytes", "h3attn_pool", "h3attn_route", "h3attn_forward",
+           "h3attn_dense_workspace_bytes", "h3attn_dense_biased", "h3attn_check", "h3attn_selftest_timeout",
+           "h3attn_strerror")
+
+
+class H3Error(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {lib().h3attn_strerror(code).decode()} ({code})")
+
+
+class Plan(ctypes.Structure):
+    _fields_ = [("H", ctypes.c_int32), ("S", ctypes.c_int32), ("d", ctypes.c_int32), ("block", ctypes.c_int32),
+                ("sparsity", ctypes.c_float), ("n_blocks", ctypes.c_int32), ("prefix_rows", ctypes.c_int32),
+                ("first_video_block", ctypes.c_int32), ("n_forced", ctypes.c_int32),
+                ("n_video_blocks", ctypes.c_int32), ("k", ctypes.c_int32)]
+
+    def __repr__(self):
+        return "Plan(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+class Penalty(ctypes.Structure):
+    _fields_ = [("strength", ctypes.c_float), ("window", ctypes.c_float), ("falloff", ctypes.c_float),
+                ("cap", ctypes.c_float)]
+
+
+DEFAULT_PENALTY = (2.0, 0.20, 0.25, 6.0)
+
+_lib = None
+_P = ctypes.c_void_p
+
+
+def lib_path() -> str:
+    return _build.LIB
+
+
+def lib():
+    """Load libh3attn.so (building it in-tree with nvcc if it is missing or stale)."""
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        PP = ctypes.POINTER(Plan)
+        L.h3attn_plan_init.argtypes = [PP, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, _P]
+        L.h3attn_plan_init.restype = ctypes.c_int
+        L.h3attn_workspace_bytes.argtypes = [PP]
+        L.h3attn_workspace_bytes.restype = ctypes.c_size_t
+        L.h3attn_pool.argtypes = [PP, _P, ctypes.c_int, ctypes.c_int, _P, _P]
+        L.h3attn_pool.restype = ctypes.c_int
+        L.h3attn_route.argtypes = [PP, _P, _P, _P, _P, ctypes.c_size_t, _P]
+        L.h3attn_route.restype = ctypes.c_int
+        L.h3attn_forward.argtypes = [PP, _P, _P, _P, _P, _P, ctypes.POINTER(Penalty), _P, _P, _P, _P,
+                                     ctypes.c_size_t, _P]
+        L.h3attn_forward.restype = ctypes.c_int
+        L.h3attn_dense_workspace_bytes.argtypes = [ctypes.c_int]
+        L.h3attn_dense_workspace_bytes.restype = ctypes.c_size_t
+        L.h3attn_dense_biased.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, _P,
+                                          ctypes.POINTER(Penalty), _P, _P, _P, ctypes.c_size_t, _P]
+        L.h3attn_dense_biased.restype = ctypes.c_int
+        L.h3attn_check.argtypes = [_P, _P]
+        L.h3attn_check.restype = ctypes.c_int
+        L.h3attn_selftest_timeout.argtypes = [_P, ctypes.c_uint32, _P]
+        L.h3attn_selftest_timeout.restype = ctypes.c_int
+        L.h3attn_strerror.argtypes = [ctypes.c_int]
+        L.h3attn_strerror.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _raise(code: int, what: str):
+    if code != OK:
+        raise H3Error(code, what)
+
+
+def _stream(stream=None) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _dptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _check_qkv(*ts):
+    for t in ts:
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous() and t.dim() == 3):
+            raise ValueError("q/k/v/o must be contiguous CUDA bf16 [H, S, d]")
+
+
+def _pen(pen) -> Optional[Penalty]:
+    if pen is None:
+        return None
+    if isinstance(pen, Penalty):
+        return pen
+    s, w, f, c = pen
+    return Penalty(s, w, f, c)
+
+
+def plan(H: int, S: int, d: int, seg_host, sparsity: float = 0.0, block: int = 64) -> Plan:
+    """Block plan from the host copy of seg (numpy or CPU tensor, uint8 [S])."""
+    seg = np.ascontiguousarray(seg_host.cpu().numpy() if isinstance(seg_host, torch.Tensor) else seg_host,
+                               dtype=np.uint8)
+    if seg.shape != (S,):
+        raise ValueError("seg must have S entries")
+    p = Plan()
+    _raise(lib().h3attn_plan_init(ctypes.byref(p), H, S, d, block, sparsity, seg.ctypes.data), "plan_init")
+    return p
+
+
+def workspace(p: Plan, device="cuda") -> torch.Tensor:
+    n = lib().h3attn_workspace_bytes(ctypes.byref(p))
+    if n == 0:
+        raise H3Error(EINVAL, "workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def dense_workspace(S: int, device="cuda") -> torch.Tensor:
+    return torch.zeros(lib().h3attn_dense_workspace_bytes(S), dtype=torch.uint8, device=device)
+
+
+def pool(p: Plan, x: torch.Tensor, first_block: int = 0, n_out: Optional[int] = None, out=None, stream=None):
+    """Block means (fp32 [H, n_out, d]) of blocks [first_block, first_block + n_out)."""
+    _check_qkv(x)
+    n_out = p.n_blocks - first_block if n_out is None else n_out
+    if out is None:
+        out = torch.empty((p.H, n_out, p.d), dtype=torch.float32, device=x.device)
+    _raise(lib().h3attn_pool(ctypes.byref(p), x.data_ptr(), first_block, n_out, out.data_ptr(), _stream(stream)),
+           "pool")
+    return out
+
+
+def route(p: Plan, q: torch.Tensor, k: torch.Tensor, ws: torch.Tensor, kv_sel=None, stream=None) -> torch.Tensor:
+    """Routed key blocks int32 [H, n_video_blocks, k] (absolute block ids, ascending)."""
+    _check_qkv(q, k)
+    if kv_sel is None:
+        kv_sel = torch.empty((p.H, p.n_video_blocks, p.k), dtype=torch.int32, device=q.device)
+    _raise(lib().h3attn_route(ctypes.byref(p), q.data_ptr(), k.data_ptr(), kv_sel.data_ptr(), ws.data_ptr(),
+                              ws.numel(), _stream(stream)), "route")
+    return kv_sel
+
+
+def forward(p: Plan, q, k, v, seg, times, pen=DEFAULT_PENALTY, kv_sel=None, ws=None, out=None,
+            lse: bool | torch.Tensor = False, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Attention over the routed tiles (kv_sel None = dense) with the temporal penalty (pen None = off)."""
+    _check_qkv(q, k, v)
+    if ws is None:
+        ws = workspace(p, q.device)
+    o = torch.empty_like(q) if out is None else out
+    lse_t = lse if isinstance(lse, torch.Tensor) else (
+        torch.empty((p.H, p.S), dtype=torch.float32, device=q.device) if lse else None)
+    pn = _pen(pen)
+    _raise(lib().h3attn_forward(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), seg.data_ptr(),
+                                _dptr(times), ctypes.byref(pn) if pn is not None else None, _dptr(kv_sel),
+                                o.data_ptr(), _dptr(lse_t), ws.data_ptr(), ws.numel(), _stream(stream)), "forward")
+    return o, lse_t
+
+
+def dense_biased(q, k, v, seg, times, pen=DEFAULT_PENALTY, ws=None, out=None, lse: bool = False, stream=None):
+    """Dense attention with the temporal penalty on output -> guide pairs."""
+    _check_qkv(q, k, v)
+    H, S, d = q.shape
+    if ws is None:
+        ws = dense_workspace(S, q.device)
+    o = torch.empty_like(q) if out is None else out
+    lse_t = torch.empty((H, S), dtype=torch.float32, device=q.device) if lse else None
+    pn = _pen(pen)
+    _raise(lib().h3attn_dense_biased(H, S, d, q.data_ptr(), k.data_ptr(), v.data_ptr(), seg.data_ptr(),
+                                     _dptr(times), ctypes.byref(pn) if pn is not None else None, o.data_ptr(),
+                                     _dptr(lse_t), ws.data_ptr(), ws.numel(), _stream(stream)), "dense_biased")
+    return o, lse_t
+
+
+def check(ws: torch.Tensor, stream=None) -> int:
+    """Synchronise and return (and clear) the device status word."""
+    return int(lib().h3attn_check(ws.data_ptr(), _stream(stream)))
+
+
+def selftest_timeout(ws: torch.Tensor, polls: int, stream=None) -> None:
+    _raise(lib().h3attn_selftest_timeout(ws.data_ptr(), polls, _stream(stream)), "selftest_timeout")

@@ -1,0 +1,293 @@
+// C ABI of libh3attn: argument validation, block plan, workspace layout,
+// TMA descriptors and kernel launches.  See include/h3attn.h for the contract.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "h3attn.h"
+#include "kernels.cuh"
+
+namespace h3 {
+size_t route_smem_bytes(int d, int n_video);
+}
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kStatusBytes = 256;
+constexpr uint32_t kWaitPolls = 0xFFFFFFFFu;
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait: far above any legitimate stall
+constexpr int kMaxSmem = 227 * 1024;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct WsLayout {
+  size_t desc, qp, kp, total;
+};
+
+WsLayout ws_layout(int H, int d, int n_blocks, int n_video) {
+  WsLayout w;
+  w.desc = kStatusBytes;
+  w.qp = w.desc + align_up((size_t)n_blocks * sizeof(uint2));
+  w.kp = w.qp + align_up((size_t)H * n_video * d * sizeof(float));
+  w.total = w.kp + align_up((size_t)H * n_video * d * sizeof(float));
+  return w;
+}
+
+bool plan_ok(const h3attn_plan* p) {
+  return p != nullptr && p->H > 0 && p->S > 0 && (p->d == 64 || p->d == 128) && p->block == h3::kBlock &&
+         p->n_blocks == (p->S + p->block - 1) / p->block && p->n_blocks <= h3::kMaxBlocks &&
+         p->first_video_block >= 0 && p->first_video_block <= p->n_blocks &&
+         p->n_video_blocks == p->n_blocks - p->first_video_block && p->n_forced == p->first_video_block &&
+         (p->n_video_blocks == 0 || (p->k >= 1 && p->k <= p->n_video_blocks));
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// bf16 [H][S][d] viewed as 3-D {d, S, H}; box {64, 64, 1}, 128-byte swizzle,
+// rows past S (and past the head) read as zero.
+bool make_map(CUtensorMap* m, const void* base, int H, int S, int d) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)S, (cuuint64_t)H};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)S * d * 2};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool finite_nonneg(float x) { return std::isfinite(x) && x >= 0.0f; }
+
+int forward_impl(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                 const uint8_t* seg, const float* times, const h3attn_penalty* pen, const int32_t* kv_sel,
+                 uint16_t* o, float* lse, void* ws, size_t ws_bytes, size_t ws_needed, cudaStream_t stream) {
+  if (!plan_ok(plan)) return H3ATTN_EINVAL;
+  if (!q || !k || !v || !seg || !o) return H3ATTN_EINVAL;
+  if (ws == nullptr || ws_bytes < ws_needed) return H3ATTN_EWORKSPACE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(ws)) return H3ATTN_EALIGN;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return H3ATTN_EALIGN;
+  bool pen_on = false;
+  if (pen != nullptr) {
+    if (!finite_nonneg(pen->strength) || !finite_nonneg(pen->window) || !finite_nonneg(pen->cap) ||
+        !std::isfinite(pen->falloff))
+      return H3ATTN_EINVAL;
+    pen_on = pen->strength > 0.0f && pen->cap > 0.0f;
+    if (pen_on && !(pen->falloff > 0.0f)) return H3ATTN_EINVAL;
+    if (pen_on && times == nullptr) return H3ATTN_EINVAL;
+  }
+  if (h3::attn_smem_bytes(plan->d, plan->n_blocks) > kMaxSmem) return H3ATTN_EUNSUPPORTED;
+  const bool routed = kv_sel != nullptr && plan->n_video_blocks > 0;
+
+  h3::AttnParams p{};
+  p.H = plan->H;
+  p.S = plan->S;
+  p.d = plan->d;
+  p.n_blocks = plan->n_blocks;
+  p.first_video_block = plan->first_video_block;
+  p.n_video_blocks = plan->n_video_blocks;
+  p.k = plan->k;
+  p.kv_sel = routed ? kv_sel : nullptr;
+  p.seg = seg;
+  p.times = times;
+  p.o = o;
+  p.lse = lse;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  p.status = reinterpret_cast<int*>(wsb);
+  p.kv_desc = reinterpret_cast<const uint2*>(wsb + kStatusBytes);
+  p.pen_on = pen_on ? 1 : 0;
+  const float log2e = 1.4426950408889634f;
+  p.scale_log2 = log2e / std::sqrt((float)plan->d);
+  if (pen_on) {
+    p.window = pen->window;
+    p.inv_falloff = 1.0f / pen->falloff;
+    p.strength_log2 = pen->strength * log2e;
+    p.cap_log2 = pen->cap * log2e;
+  }
+  p.wait_polls = kWaitPolls;
+  p.wait_ns = kWaitNs;
+  const int n_qtiles = (plan->n_blocks + 1) / 2;
+  p.n_dense_tiles = routed ? (plan->first_video_block + 1) / 2 : n_qtiles;
+  if (p.n_dense_tiles > n_qtiles) p.n_dense_tiles = n_qtiles;
+
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, plan->H, plan->S, plan->d) || !make_map(&tk, k, plan->H, plan->S, plan->d) ||
+      !make_map(&tv, v, plan->H, plan->S, plan->d))
+    return H3ATTN_ECUDA;
+  if (h3::launch_kv_desc(seg, pen_on ? times : nullptr, plan->S, plan->n_blocks,
+                         reinterpret_cast<uint2*>(wsb + kStatusBytes), stream) != cudaSuccess)
+    return H3ATTN_ECUDA;
+  if (h3::launch_attn(tq, tk, tv, p, n_qtiles * plan->H, stream) != cudaSuccess) return H3ATTN_ECUDA;
+  return H3ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int h3attn_plan_init(h3attn_plan* plan, int H, int S, int d, int block, float sparsity, const uint8_t* seg_host) {
+  if (plan == nullptr || seg_host == nullptr || H <= 0 || S <= 0) return H3ATTN_EINVAL;
+  if (!(sparsity >= 0.0f && sparsity < 1.0f)) return H3ATTN_EINVAL;
+  if (!(d == 64 || d == 128) || block != h3::kBlock) return H3ATTN_EUNSUPPORTED;
+  const int n_blocks = (S + block - 1) / block;
+  if (n_blocks > h3::kMaxBlocks) return H3ATTN_EUNSUPPORTED;
+  int prefix = 0;
+  while (prefix < S && seg_host[prefix] != H3ATTN_SEG_GUIDE && seg_host[prefix] != H3ATTN_SEG_OUTPUT) ++prefix;
+  for (int r = prefix; r < S; ++r)
+    if (seg_host[r] != H3ATTN_SEG_GUIDE && seg_host[r] != H3ATTN_SEG_OUTPUT) return H3ATTN_EUNSUPPORTED;
+  for (int r = 0; r < S; ++r)
+    if (seg_host[r] > H3ATTN_SEG_OUTPUT) return H3ATTN_EINVAL;
+  h3attn_plan p{};
+  p.H = H;
+  p.S = S;
+  p.d = d;
+  p.block = block;
+  p.sparsity = sparsity;
+  p.n_blocks = n_blocks;
+  p.prefix_rows = prefix;
+  p.first_video_block = (prefix + block - 1) / block;
+  p.n_forced = p.first_video_block;
+  p.n_video_blocks = n_blocks - p.first_video_block;
+  if (p.n_video_blocks > 0) {
+    const double want = std::ceil((1.0 - (double)sparsity) * (double)p.n_video_blocks - 1e-9);
+    int kk = (int)want;
+    if (kk < 1) kk = 1;
+    if (kk > p.n_video_blocks) kk = p.n_video_blocks;
+    p.k = kk;
+  } else {
+    p.k = 0;
+  }
+  *plan = p;
+  return H3ATTN_OK;
+}
+
+size_t h3attn_workspace_bytes(const h3attn_plan* plan) {
+  if (!plan_ok(plan)) return 0;
+  return ws_layout(plan->H, plan->d, plan->n_blocks, plan->n_video_blocks).total;
+}
+
+int h3attn_pool(const h3attn_plan* plan, const uint16_t* x, int first_block, int n_out, float* out, void* stream) {
+  if (!plan_ok(plan) || x == nullptr || out == nullptr) return H3ATTN_EINVAL;
+  if (first_block < 0 || n_out < 0 || first_block + n_out > plan->n_blocks) return H3ATTN_EINVAL;
+  if (!aligned16(x) || !aligned16(out)) return H3ATTN_EALIGN;
+  if (n_out == 0) return H3ATTN_OK;
+  if (h3::launch_pool(x, out, nullptr, nullptr, plan->H, plan->S, plan->d, first_block, n_out,
+                      static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return H3ATTN_ECUDA;
+  return H3ATTN_OK;
+}
+
+int h3attn_route(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, int32_t* kv_sel, void* ws,
+                 size_t ws_bytes, void* stream) {
+  if (!plan_ok(plan) || q == nullptr || k == nullptr || kv_sel == nullptr) return H3ATTN_EINVAL;
+  if (plan->n_video_blocks == 0) return H3ATTN_EINVAL;
+  const WsLayout w = ws_layout(plan->H, plan->d, plan->n_blocks, plan->n_video_blocks);
+  if (ws == nullptr || ws_bytes < w.total) return H3ATTN_EWORKSPACE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(ws) || (reinterpret_cast<uintptr_t>(kv_sel) & 3u))
+    return H3ATTN_EALIGN;
+  if (h3::route_smem_bytes(plan->d, plan->n_video_blocks) > (size_t)kMaxSmem) return H3ATTN_EUNSUPPORTED;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  float* qp = reinterpret_cast<float*>(wsb + w.qp);
+  float* kp = reinterpret_cast<float*>(wsb + w.kp);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (h3::launch_pool(q, qp, k, kp, plan->H, plan->S, plan->d, plan->first_video_block, plan->n_video_blocks, st) !=
+      cudaSuccess)
+    return H3ATTN_ECUDA;
+  if (h3::launch_route(qp, kp, kv_sel, plan->H, plan->d, plan->n_video_blocks, plan->k, plan->first_video_block,
+                       st) != cudaSuccess)
+    return H3ATTN_ECUDA;
+  return H3ATTN_OK;
+}
+
+int h3attn_forward(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                   const uint8_t* seg, const float* times, const h3attn_penalty* pen, const int32_t* kv_sel,
+                   uint16_t* o, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  if (!plan_ok(plan)) return H3ATTN_EINVAL;
+  const size_t need = kStatusBytes + align_up((size_t)plan->n_blocks * sizeof(uint2));
+  if (kv_sel != nullptr && (reinterpret_cast<uintptr_t>(kv_sel) & 3u)) return H3ATTN_EALIGN;
+  return forward_impl(plan, q, k, v, seg, times, pen, kv_sel, o, lse, ws, ws_bytes, need,
+                      static_cast<cudaStream_t>(stream));
+}
+
+size_t h3attn_dense_workspace_bytes(int S) {
+  if (S <= 0) return 0;
+  const int n_blocks = (S + h3::kBlock - 1) / h3::kBlock;
+  return kStatusBytes + align_up((size_t)n_blocks * sizeof(uint2));
+}
+
+int h3attn_dense_biased(int H, int S, int d, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                        const uint8_t* seg, const float* times, const h3attn_penalty* pen, uint16_t* o, float* lse,
+                        void* ws, size_t ws_bytes, void* stream) {
+  if (H <= 0 || S <= 0) return H3ATTN_EINVAL;
+  if (!(d == 64 || d == 128)) return H3ATTN_EUNSUPPORTED;
+  h3attn_plan p{};
+  p.H = H;
+  p.S = S;
+  p.d = d;
+  p.block = h3::kBlock;
+  p.sparsity = 0.0f;
+  p.n_blocks = (S + h3::kBlock - 1) / h3::kBlock;
+  if (p.n_blocks > h3::kMaxBlocks) return H3ATTN_EUNSUPPORTED;
+  p.prefix_rows = S;
+  p.first_video_block = p.n_blocks;
+  p.n_forced = p.n_blocks;
+  p.n_video_blocks = 0;
+  p.k = 0;
+  return forward_impl(&p, q, k, v, seg, times, pen, nullptr, o, lse, ws, ws_bytes, h3attn_dense_workspace_bytes(S),
+                      static_cast<cudaStream_t>(stream));
+}
+
+int h3attn_check(void* ws, void* stream) {
+  if (ws == nullptr) return H3ATTN_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return H3ATTN_ECUDA;
+  int status = 0;
+  if (cudaMemcpy(&status, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return H3ATTN_ECUDA;
+  if (status != 0 && cudaMemset(ws, 0, sizeof(int)) != cudaSuccess) return H3ATTN_ECUDA;
+  if (status == h3::kStatusTimeout) return H3ATTN_ETIMEOUT;
+  if (status == h3::kStatusData) return H3ATTN_EDATA;
+  return status == 0 ? H3ATTN_OK : H3ATTN_ECUDA;
+}
+
+int h3attn_selftest_timeout(void* ws, uint32_t polls, void* stream) {
+  if (ws == nullptr || !aligned16(ws)) return H3ATTN_EINVAL;
+  if (h3::launch_selftest_timeout(static_cast<int*>(ws), polls, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return H3ATTN_ECUDA;
+  return H3ATTN_OK;
+}
+
+const char* h3attn_strerror(int status) {
+  switch (status) {
+    case H3ATTN_OK: return "ok";
+    case H3ATTN_EINVAL: return "invalid argument";
+    case H3ATTN_EUNSUPPORTED: return "unsupported shape or layout";
+    case H3ATTN_EALIGN: return "pointer not aligned (16 bytes for tensors and workspace)";
+    case H3ATTN_ECUDA: return "CUDA call or kernel launch failed";
+    case H3ATTN_ETIMEOUT: return "a bounded device-side wait gave up";
+    case H3ATTN_EWORKSPACE: return "workspace missing or too small";
+    case H3ATTN_EDATA: return "routed list holds a block index outside the video key blocks";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,54 @@
+// Internal interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace h3 {
+
+constexpr int kSegGuide = 3;
+constexpr int kSegOutput = 4;
+constexpr int kBlock = 64;
+constexpr int kMaxBlocks = 8192;  // S <= 524288: one 16-bit block id, lists fit in shared memory
+
+// device status word values (the C ABI maps them to H3ATTN_E*)
+constexpr int kStatusTimeout = 1;
+constexpr int kStatusData = 2;
+
+struct AttnParams {
+  int H, S, d;
+  int n_blocks, first_video_block, n_video_blocks, k;
+  int n_dense_tiles;           // query tiles holding a dense query block (scheduled first)
+  const int32_t* kv_sel;       // [H][nV][k] or null (dense)
+  const uint8_t* seg;          // [S]
+  const float* times;          // [S]
+  const uint2* kv_desc;        // [n_blocks]: x = valid rows | kind << 8, y = time bits (kind 1)
+  uint16_t* o;                 // bf16 [H][S][d]
+  float* lse;                  // [H][S] or null
+  int* status;                 // device status word
+  int pen_on;
+  float scale_log2;            // log2(e) / sqrt(d)
+  float window, inv_falloff, strength_log2, cap_log2;
+  uint32_t wait_polls;         // bounded waits: poll budget
+  uint64_t wait_ns;            // bounded waits: time budget
+};
+
+int attn_smem_bytes(int d, int n_blocks);
+cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                        const AttnParams& p, int n_ctas, cudaStream_t stream);
+
+// kv_desc[b] for every key block (valid rows, guide-key kind, uniform time)
+cudaError_t launch_kv_desc(const uint8_t* seg, const float* times, int S, int n_blocks, uint2* kv_desc,
+                           cudaStream_t stream);
+
+// mean-pool blocks [first_block, first_block + n_out) of up to two bf16 [H][S][d] tensors
+cudaError_t launch_pool(const uint16_t* x0, float* out0, const uint16_t* x1, float* out1, int H, int S,
+                        int d, int first_block, int n_out, cudaStream_t stream);
+
+// pooled scores of video query blocks vs video key blocks + top-k, per head
+cudaError_t launch_route(const float* qp, const float* kp, int32_t* kv_sel, int H, int d, int n_video,
+                         int k, int first_video_block, cudaStream_t stream);
+
+cudaError_t launch_selftest_timeout(int* status, uint32_t polls, cudaStream_t stream);
+
+}  // namespace h3

@@ -1,0 +1,179 @@
+/*
+ * h3attn — biased, block-routed attention over MiniMax-H3's packed sequence
+ * [text | image-ref | audio | guide video | output video], on one B200
+ * (sm_100a).  Plain C ABI: pointers and sizes only.
+ *
+ * Operation (sources are web pages, cited by title and section):
+ *
+ *  Routing — "H3 SLA Attention" node page, "How it works": Q and K are
+ *  mean-pooled per 64-row block ("pooled centroids"), every video query block
+ *  is scored against every video key block with one small pooled matmul, and
+ *  only the top (1 - sparsity_ratio) fraction of those key blocks is attended.
+ *  Its inputs table: protect_audio always attends the blocks overlapping text,
+ *  conditioning and audio rows; block_size 64.  "Per-layer attention config
+ *  LoRAs", "Experimental: audio/text protection": prefix keys stay exact
+ *  (sink_keys "prefix") and audio queries stay fully exact (sink_queries
+ *  "audio").  "H3 sparse-attention breakpoints", "Results at a glance": the
+ *  kept fraction counts the available video key/value tiles only.
+ *
+ *  Attention — "Flash Partitions for H3 native temporal alignment", section 1
+ *  "What receives the temporal bias?": for an output-video query and a
+ *  guide-video key,
+ *     dt = |t_q - t_k|,
+ *     penalty(dt) = min(strength * (max(dt - window, 0) / falloff)^2, cap),
+ *     score = q.k / sqrt(head_dim) - penalty(dt);
+ *  every other pair keeps score = q.k / sqrt(head_dim).  Defaults: strength
+ *  2.0, window 0.20 s, falloff 0.25 s, cap 6.0 (same page; also "TARA :
+ *  alignement temporel natif ...", "La règle temporelle").  The output is the
+ *  exact softmax-weighted sum of V over the attended keys; LSE is the
+ *  natural-log normaliser (same page, section 4).
+ *
+ * Readings where the pages are silent: pooled score = Qp.Kp / sqrt(d), per
+ * head; k = clamp(ceil((1 - s) * nV - 1e-9), 1, nV); ties go to the lower
+ * block index; a key block is forced and a query block is dense iff it holds
+ * any non-video row; dropped blocks leave the softmax; routing ignores the
+ * penalty, which is applied exactly on the routed output -> guide pairs.
+ *
+ * Conventions for every call:
+ *  - Q, K, V, O are bf16 (passed as uint16_t bit patterns), layout
+ *    [H][S][d], contiguous, row-major, on the device; base addresses 16-byte
+ *    aligned.  seg is uint8 [S] and times is float32 [S] (seconds), on the
+ *    device; times are read only for guide/output rows.
+ *  - The caller owns every buffer; the library allocates no memory.
+ *  - All device work is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream).  Only h3attn_check synchronises.
+ *  - Return value 0 on success, a negative H3ATTN_E* code otherwise.  On a
+ *    host-side error nothing is launched and outputs are untouched.  Device-
+ *    side failures (a bounded wait that ran out, a corrupt routed list) are
+ *    recorded in the workspace status word and reported by h3attn_check.
+ *  - No call prints, aborts or throws.
+ */
+#ifndef H3ATTN_H
+#define H3ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define H3ATTN_API __attribute__((visibility("default")))
+#else
+#define H3ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define H3ATTN_OK 0
+#define H3ATTN_EINVAL (-1)       /* bad argument: null pointer, bad size, bad value */
+#define H3ATTN_EUNSUPPORTED (-2) /* d not 64/128, block not 64, video rows not a suffix, S too large */
+#define H3ATTN_EALIGN (-3)       /* a base address is not 16-byte aligned */
+#define H3ATTN_ECUDA (-4)        /* a CUDA runtime/driver call or launch failed */
+#define H3ATTN_ETIMEOUT (-5)     /* a bounded device-side wait gave up */
+#define H3ATTN_EWORKSPACE (-6)   /* workspace missing or too small */
+#define H3ATTN_EDATA (-7)        /* device found a corrupt routed list (index out of range) */
+
+/* Segment ids of the packed sequence. */
+enum {
+  H3ATTN_SEG_TEXT = 0,
+  H3ATTN_SEG_IMAGE_REF = 1,
+  H3ATTN_SEG_AUDIO = 2,
+  H3ATTN_SEG_GUIDE = 3,
+  H3ATTN_SEG_OUTPUT = 4
+};
+
+/* Temporal penalty controls ("Flash Partitions ...", section 1).
+ * strength >= 0, window >= 0, falloff > 0, cap >= 0, all finite.
+ * strength == 0 or cap == 0 removes the penalty (same page, section 4). */
+typedef struct {
+  float strength;
+  float window;  /* seconds */
+  float falloff; /* seconds */
+  float cap;
+} h3attn_penalty;
+
+/* Block plan of one packed sequence.  Plain data, caller-owned, filled by
+ * h3attn_plan_init (host only, no CUDA call).
+ *  n_blocks          ceil(S / block)
+ *  prefix_rows       rows before the first video row (video rows are a suffix)
+ *  first_video_block first block whose rows are all video = ceil(prefix_rows / block)
+ *  n_forced          = first_video_block: key blocks always attended, and
+ *                    query blocks attended densely (they hold a non-video row)
+ *  n_video_blocks    n_blocks - first_video_block (nV)
+ *  k                 routed video key blocks per video query block */
+typedef struct {
+  int32_t H, S, d, block;
+  float sparsity;
+  int32_t n_blocks, prefix_rows, first_video_block, n_forced, n_video_blocks, k;
+} h3attn_plan;
+
+/* Fill *plan from the host copy of seg[S].  block must be 64; d 64 or 128;
+ * 0 <= sparsity < 1; rows with seg 3/4 (video) must form a contiguous suffix
+ * of the sequence ("Flash Partitions ...", section 7: contiguous video rows).
+ * A sequence without video rows is accepted (no routing; everything dense). */
+H3ATTN_API int h3attn_plan_init(h3attn_plan* plan, int H, int S, int d, int block, float sparsity,
+                     const uint8_t* seg_host);
+
+/* Bytes of device workspace a plan needs for h3attn_route and h3attn_forward
+ * (status word, per-block key descriptors, pooled Q and K of the video blocks).
+ * The caller allocates it once, zero-filled (the first 256 bytes hold the
+ * status word that h3attn_check reads and clears). */
+H3ATTN_API size_t h3attn_workspace_bytes(const h3attn_plan* plan);
+
+/* Block mean-pool of one tensor ("H3 SLA Attention", pooled centroids):
+ * out[h][b - first_block][c] = mean over the valid rows r of block b
+ * (rows [b*64, min(S, b*64+64))) of x[h][r][c], accumulated in fp32.
+ * x: bf16 [H][S][d] device; out: float32 [H][n_out][d] device;
+ * blocks [first_block, first_block + n_out) must lie in [0, n_blocks). */
+H3ATTN_API int h3attn_pool(const h3attn_plan* plan, const uint16_t* x, int first_block, int n_out, float* out,
+                void* stream);
+
+/* Routing (pool + pooled score + top-k).  For every head h and video query
+ * block i (block first_video_block + i):
+ *   kv_sel[h][i][0..k) = the k video key blocks j with the highest
+ *   Qp[h][i].Kp[h][j] / sqrt(d) (fp32), ties to the lower block, listed as
+ *   absolute block indices in ascending order.
+ * q, k: bf16 [H][S][d] device; kv_sel: int32 [H][n_video_blocks][k] device.
+ * ws: workspace of at least h3attn_workspace_bytes(plan) bytes. */
+H3ATTN_API int h3attn_route(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, int32_t* kv_sel,
+                 void* ws, size_t ws_bytes, void* stream);
+
+/* Exact attention over the routed tiles with the temporal penalty.
+ * Each query row attends: all keys if its block is a forced (non-video)
+ * block or kv_sel is NULL; otherwise the forced key blocks plus the routed
+ * blocks kv_sel[h][qblock - first_video_block][0..k).  pen NULL = no penalty.
+ * o: bf16 [H][S][d] device (rounded to nearest even); lse: float32 [H][S]
+ * device natural-log normaliser, or NULL.
+ * Routed indices outside [first_video_block, n_blocks) are ignored and flagged
+ * (H3ATTN_EDATA from h3attn_check). */
+H3ATTN_API int h3attn_forward(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                   const uint8_t* seg, const float* times, const h3attn_penalty* pen,
+                   const int32_t* kv_sel, uint16_t* o, float* lse, void* ws, size_t ws_bytes,
+                   void* stream);
+
+/* Dense biased attention (every query attends every key; the penalty on
+ * output -> guide pairs): h3attn_forward with a dense plan and kv_sel NULL.
+ * Needs h3attn_dense_workspace_bytes(S) bytes of zero-filled workspace. */
+H3ATTN_API size_t h3attn_dense_workspace_bytes(int S);
+H3ATTN_API int h3attn_dense_biased(int H, int S, int d, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                        const uint8_t* seg, const float* times, const h3attn_penalty* pen, uint16_t* o,
+                        float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, then return and clear the device-side status word
+ * of ws: H3ATTN_OK, H3ATTN_ETIMEOUT or H3ATTN_EDATA; H3ATTN_ECUDA if the
+ * stream reports an error. */
+H3ATTN_API int h3attn_check(void* ws, void* stream);
+
+/* Self-test of the bounded-wait mechanism: launches one block that waits on
+ * an mbarrier nothing arrives at, with a limit of `polls` polls, and records
+ * H3ATTN_ETIMEOUT in the status word when it gives up.  No other work. */
+H3ATTN_API int h3attn_selftest_timeout(void* ws, uint32_t polls, void* stream);
+
+/* Static description of a status code (never NULL). */
+H3ATTN_API const char* h3attn_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* H3ATTN_H */

@@ -1,0 +1,123 @@
+"""C-ABI library: loads without a GPU, exports every declared symbol, host-side
+plan logic and argument validation (no device work)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import biased_attention_video_b200 as h3
+import inputs
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "h3attn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(h3attn_[a-z_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    path = h3.lib_path()
+    h3.lib()
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (h3attn_\w+)", out))
+    decl = declared_functions()
+    assert decl, "no declarations parsed"
+    assert set(decl) <= exported, set(decl) - exported
+    assert set(decl) == set(h3.EXPORTS)
+    for name in decl:
+        getattr(h3.lib(), name)
+
+
+def test_library_targets_sm100a():
+    out = subprocess.run(["/usr/local/cuda/bin/cuobjdump", "--list-elf", h3.lib_path()], capture_output=True,
+                         text=True).stdout
+    assert "sm_100a" in out
+
+
+@pytest.mark.parametrize("c", [1, 2, 3, 4, 5])
+def test_plan_matches_oracle_block_classes(c):
+    cfg = inputs.CONFIGS[c]
+    seg, _, _ = cfg.layout()
+    for s in cfg.sparsities:
+        p = h3.plan(cfg.H, cfg.S, cfg.d, seg, sparsity=s)
+        cls = oracle.block_classes(seg)
+        assert p.n_blocks == len(cls)
+        assert p.first_video_block == p.n_forced == int(cls.sum())
+        assert np.all(cls[:p.first_video_block] == 1) and np.all(cls[p.first_video_block:] == 0)
+        assert p.n_video_blocks == len(cls) - int(cls.sum())
+        if p.n_video_blocks:
+            assert p.k == oracle.k_for(p.n_video_blocks, s)
+
+
+def test_plan_known_values():
+    seg5, _, _ = inputs.CONFIGS[5].layout()
+    p = h3.plan(56, 116883, 128, seg5, sparsity=0.90)
+    assert (p.n_blocks, p.first_video_block, p.n_video_blocks, p.k, p.prefix_rows) == (1827, 33, 1794, 180, 2079)
+    seg2, _, _ = inputs.CONFIGS[2].layout()
+    p2 = h3.plan(8, 16384, 128, seg2, sparsity=0.85)
+    assert (p2.n_blocks, p2.first_video_block, p2.n_video_blocks, p2.k) == (256, 10, 246, 37)
+
+
+def test_plan_rejects_bad_arguments():
+    seg = np.array([0] * 10 + [4] * 100, np.uint8)
+    with pytest.raises(h3.H3Error) as e:
+        h3.plan(2, 110, 96, seg)
+    assert e.value.code == h3.EUNSUPPORTED
+    with pytest.raises(h3.H3Error) as e:
+        h3.plan(2, 110, 128, seg, sparsity=1.0)
+    assert e.value.code == h3.EINVAL
+    with pytest.raises(h3.H3Error) as e:
+        h3.plan(2, 110, 128, seg, block=128)
+    assert e.value.code == h3.EUNSUPPORTED
+    bad = seg.copy()
+    bad[50] = 2  # audio row inside the video suffix
+    with pytest.raises(h3.H3Error) as e:
+        h3.plan(2, 110, 128, bad)
+    assert e.value.code == h3.EUNSUPPORTED
+    bad = seg.copy()
+    bad[3] = 9
+    with pytest.raises(h3.H3Error) as e:
+        h3.plan(2, 110, 128, bad)
+    assert e.value.code == h3.EINVAL
+
+
+def test_plan_without_video_is_dense():
+    seg = np.zeros(300, np.uint8)
+    p = h3.plan(1, 300, 64, seg)
+    assert p.n_video_blocks == 0 and p.first_video_block == p.n_blocks == 5 and p.k == 0
+
+
+def test_host_validation_before_any_device_work():
+    L = h3.lib()
+    seg = np.array([0] * 64 + [4] * 192, np.uint8)
+    p = h3.plan(1, 256, 128, seg, sparsity=0.5)
+    # null tensors
+    assert L.h3attn_forward(ctypes.byref(p), None, None, None, None, None, None, None, None, None, None, 0,
+                            None) == h3.EINVAL
+    fake = 1 << 40  # never dereferenced: validation fails first
+    ws_need = L.h3attn_workspace_bytes(ctypes.byref(p))
+    assert ws_need > 0
+    assert L.h3attn_forward(ctypes.byref(p), fake, fake, fake, fake, fake, None, None, fake, None, fake, 16,
+                            None) == h3.EWORKSPACE
+    assert L.h3attn_forward(ctypes.byref(p), fake + 2, fake, fake, fake, fake, None, None, fake, None, fake,
+                            ws_need, None) == h3.EALIGN
+    bad_pen = h3.Penalty(2.0, 0.2, 0.0, 6.0)  # falloff 0 with the penalty on
+    assert L.h3attn_forward(ctypes.byref(p), fake, fake, fake, fake, fake, ctypes.byref(bad_pen), None, fake, None,
+                            fake, ws_need, None) == h3.EINVAL
+    nan_pen = h3.Penalty(float("nan"), 0.2, 0.25, 6.0)
+    assert L.h3attn_forward(ctypes.byref(p), fake, fake, fake, fake, fake, ctypes.byref(nan_pen), None, fake, None,
+                            fake, ws_need, None) == h3.EINVAL
+    assert L.h3attn_route(ctypes.byref(p), fake, fake, fake, fake, 8, None) == h3.EWORKSPACE
+    assert L.h3attn_pool(ctypes.byref(p), fake, 2, 9, fake, None) == h3.EINVAL
+    assert L.h3attn_dense_biased(1, 256, 80, fake, fake, fake, fake, fake, None, fake, None, fake, 1 << 20,
+                                 None) == h3.EUNSUPPORTED
+    p.k = 0  # corrupt plan
+    assert L.h3attn_workspace_bytes(ctypes.byref(p)) == 0
+    for code in [0, -1, -2, -3, -4, -5, -6, -7, -99]:
+        assert isinstance(L.h3attn_strerror(code), bytes)

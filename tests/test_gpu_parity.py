@@ -1,0 +1,223 @@
+"""GPU parity against the fp64 oracle, through the C ABI (libh3attn)."""
+import numpy as np
+import pytest
+import torch
+
+import biased_attention_video_b200 as h3
+import inputs
+import oracle
+from parity import (LSE_ABS, compare_outputs, compare_routing, dev_bf16, host_bits, make, sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+PEN = inputs.DEFAULT_PENALTY
+
+
+def _layout(text, audio, gframes, gtok, oframes, otok):
+    segs = [inputs.Segment(inputs.SEG_TEXT, text)] if text else []
+    if audio:
+        segs.append(inputs.Segment(inputs.SEG_AUDIO, audio))
+    if gframes:
+        segs.append(inputs.Segment(inputs.SEG_GUIDE, gframes * gtok, gframes))
+    if oframes:
+        segs.append(inputs.Segment(inputs.SEG_OUTPUT, oframes * otok, oframes))
+    return segs
+
+
+# ------------------------------------------------------------------ pooling
+
+@pytest.mark.parametrize("d,segs", [
+    (128, _layout(256, 384, 0, 0, 41, 384)),           # config-2 packing
+    (64, _layout(20, 30, 3, 37, 3, 41)),               # ragged tail (S = 284)
+    (128, _layout(1, 0, 0, 0, 0, 0)),                  # S = 1
+])
+def test_pool_matches_oracle(d, segs):
+    cfg = inputs.custom(3, d, segs, seed=21, cluster_norm=2.0)
+    x = make(cfg)
+    seg = x["seg"]
+    p = h3.plan(cfg.H, cfg.S, d, seg)
+    got = h3.pool(p, x["k_d"]).cpu().numpy()
+    ref = oracle.pool(x["k"])
+    assert got.shape == ref.shape
+    assert np.abs(got - ref).max() <= 1e-6 * max(1.0, np.abs(ref).max())
+    if p.n_blocks > 2:
+        part = h3.pool(p, x["q_d"], first_block=1, n_out=p.n_blocks - 2).cpu().numpy()
+        assert np.abs(part - oracle.pool(x["q"])[:, 1:-1]).max() <= 1e-6 * max(1.0, np.abs(ref).max())
+
+
+# ------------------------------------------------------------------ routing
+
+def _route_and_compare(cfg, sparsity, heads=None):
+    x = make(cfg)
+    p = h3.plan(cfg.H, cfg.S, cfg.d, x["seg"], sparsity=sparsity)
+    ws = h3.workspace(p)
+    sel = h3.route(p, x["q_d"], x["k_d"], ws).cpu().numpy()
+    assert h3.check(ws) == h3.OK
+    heads = list(range(cfg.H)) if heads is None else heads
+    ref, scores, kth = oracle.route(x["q"][heads], x["k"][heads], x["seg"], sparsity, want_scores=True)
+    compare_routing(sel[heads], ref, scores, kth, p.first_video_block, cfg.name)
+    return p, x, sel, ws
+
+
+def test_route_config2():
+    _route_and_compare(inputs.CONFIGS[2], 0.85)
+
+
+@pytest.mark.parametrize("sparsity", [0.0, 0.60, 0.85, 0.90])
+def test_route_config3_sampled_heads(sparsity):
+    _route_and_compare(inputs.CONFIGS[3], sparsity, heads=[0, 27, 55])
+
+
+def test_route_tie_goes_to_lower_block():
+    segs = _layout(64, 0, 0, 0, 8, 64)
+    cfg = inputs.custom(2, 128, segs, seed=5, cluster_norm=2.0)
+    x = make(cfg, device=None)
+    k = x["k"].copy()
+    k[:, 4 * 64:5 * 64] = k[:, 7 * 64:8 * 64]      # blocks 4 and 7 score identically
+    p = h3.plan(2, cfg.S, 128, x["seg"], sparsity=0.5)
+    ws = h3.workspace(p)
+    sel = h3.route(p, dev_bf16(x["q"]), dev_bf16(k), ws).cpu().numpy()
+    ref, _, _ = oracle.route(x["q"], k, x["seg"], 0.5)
+    assert np.array_equal(sel, ref)
+
+
+# ---------------------------------------------------------------- attention
+
+def _forward_all_rows(cfg, sparsity, pen, routed=True, lse=True):
+    x = make(cfg)
+    p = h3.plan(cfg.H, cfg.S, cfg.d, x["seg"], sparsity=sparsity)
+    ws = h3.workspace(p)
+    sel_d = None
+    sel = None
+    if routed and p.n_video_blocks > 0:
+        sel_d = h3.route(p, x["q_d"], x["k_d"], ws)
+        sel = sel_d.cpu().numpy()
+        ref_sel, scores, kth = oracle.route(x["q"], x["k"], x["seg"], sparsity, want_scores=True)
+        compare_routing(sel, ref_sel, scores, kth, p.first_video_block, cfg.name)
+    o, l = h3.forward(p, x["q_d"], x["k_d"], x["v_d"], x["seg_d"], x["times_d"], pen=pen, kv_sel=sel_d, ws=ws,
+                      lse=lse)
+    assert h3.check(ws) == h3.OK
+    ref_o, ref_l = oracle.attend(x["q"], x["k"], x["v"], x["seg"], x["times"], pen=pen, sel=sel)
+    H, S, d = x["q"].shape
+    compare_outputs(host_bits(o).reshape(H * S, d), ref_o, cfg.name)
+    if lse:
+        assert np.abs(l.cpu().numpy().reshape(-1) - ref_l).max() <= LSE_ABS
+    return x, p
+
+
+RAGGED = [
+    (128, _layout(0, 0, 0, 0, 1, 1)),            # S = 1
+    (128, _layout(10, 0, 1, 20, 1, 33)),         # S = 63
+    (64, _layout(10, 5, 1, 25, 1, 25)),          # S = 65
+    (128, _layout(0, 7, 2, 30, 2, 30)),          # S = 127
+    (64, _layout(9, 0, 2, 30, 2, 30)),           # S = 129
+    (128, _layout(20, 30, 3, 37, 3, 41)),        # S = 284
+    (128, _layout(64, 160, 5, 100, 5, 110)),     # S = 1274
+]
+
+
+@pytest.mark.parametrize("d,segs", RAGGED)
+@pytest.mark.parametrize("pen", [None, PEN])
+def test_forward_dense_ragged(d, segs, pen):
+    cfg = inputs.custom(2, d, segs, seed=33, cluster_norm=0.0)
+    _forward_all_rows(cfg, 0.0, pen, routed=False)
+
+
+@pytest.mark.parametrize("d,segs", RAGGED[4:])
+@pytest.mark.parametrize("sparsity", [0.5, 0.8])
+def test_forward_routed_ragged(d, segs, sparsity):
+    cfg = inputs.custom(2, d, segs, seed=44, cluster_norm=2.0)
+    _forward_all_rows(cfg, sparsity, PEN, routed=True)
+
+
+def test_config1_dense_biased():
+    cfg = inputs.CONFIGS[1]
+    x = make(cfg)
+    o, l = h3.dense_biased(x["q_d"], x["k_d"], x["v_d"], x["seg_d"], x["times_d"], pen=PEN, lse=True)
+    torch.cuda.synchronize()
+    ref_o, ref_l = oracle.attend(x["q"], x["k"], x["v"], x["seg"], x["times"], pen=PEN)
+    H, S, d = x["q"].shape
+    compare_outputs(host_bits(o).reshape(H * S, d), ref_o, cfg.name)
+    assert np.abs(l.cpu().numpy().reshape(-1) - ref_l).max() <= LSE_ABS
+    # same numbers through the planned entry point at sparsity 0
+    _forward_all_rows(cfg, 0.0, PEN, routed=True)
+
+
+def test_peaked_scores_config1():
+    """Q x 4 makes the softmax peaked (max-abs binding), still within tolerance."""
+    cfg = inputs.CONFIGS[1]
+    x = make(cfg, device=None)
+    qf = inputs.bf16_bits_to_f64(x["q"]) * 4.0
+    q4 = inputs.f32_to_bf16_bits(qf.astype(np.float32)).reshape(x["q"].shape)
+    o, _ = h3.dense_biased(dev_bf16(q4), dev_bf16(x["k"]), dev_bf16(x["v"]), torch.from_numpy(x["seg"]).cuda(),
+                           torch.from_numpy(x["times"]).cuda(), pen=PEN)
+    ref_o, _ = oracle.attend(q4, x["k"], x["v"], x["seg"], x["times"], pen=PEN)
+    H, S, d = x["q"].shape
+    compare_outputs(host_bits(o).reshape(H * S, d), ref_o, "config 1 peaked")
+
+
+def _sampled_forward(cfg, sparsity, pen, heads, blocks, x=None):
+    x = make(cfg) if x is None else x
+    p = h3.plan(cfg.H, cfg.S, cfg.d, x["seg"], sparsity=sparsity)
+    ws = h3.workspace(p)
+    sel_d = h3.route(p, x["q_d"], x["k_d"], ws) if sparsity > 0 else None
+    o, l = h3.forward(p, x["q_d"], x["k_d"], x["v_d"], x["seg_d"], x["times_d"], pen=pen, kv_sel=sel_d, ws=ws,
+                      lse=True)
+    assert h3.check(ws) == h3.OK
+    sel = None
+    if sel_d is not None:
+        sel = sel_d.cpu().numpy()[heads]
+        ref_sel, scores, kth = oracle.route(x["q"][heads], x["k"][heads], x["seg"], sparsity, want_scores=True)
+        compare_routing(sel, ref_sel, scores, kth, p.first_video_block, cfg.name)
+    rows = sample_rows(cfg.S, blocks)
+    hh = np.repeat(np.arange(len(heads)), len(rows))
+    rr = np.tile(rows, len(heads))
+    ref_o, ref_l = oracle.attend(x["q"][heads], x["k"][heads], x["v"][heads], x["seg"], x["times"], pen=pen,
+                                 sel=sel, heads=hh, rows=rr)
+    og = host_bits(o)[heads][:, rows].reshape(-1, cfg.d)
+    compare_outputs(og, ref_o, cfg.name)
+    lg = l.cpu().numpy()[heads][:, rows].reshape(-1)
+    assert np.abs(lg - ref_l).max() <= LSE_ABS
+    return x, p
+
+
+def test_config2_routed():
+    cfg = inputs.CONFIGS[2]
+    _sampled_forward(cfg, 0.85, None, heads=list(range(8)), blocks=[0, 5, 9, 10, 11, 100, 200, 255])
+
+
+@pytest.mark.parametrize("sparsity", [0.0, 0.90])
+def test_config3_sampled(sparsity):
+    cfg = inputs.CONFIGS[3]
+    _sampled_forward(cfg, sparsity, None, heads=[0, 31, 55], blocks=[0, 25, 26, 27, 28, 300, 600, 767])
+
+
+@pytest.mark.parametrize("c", [4, 5])
+def test_full_size_sampled(c):
+    """S = 116,883, H = 56, d = 128: forced/mixed block 32, first video block 33,
+    the guide/output boundary block 929, frame-straddling blocks and the 19-row tail."""
+    cfg = inputs.CONFIGS[c]
+    _sampled_forward(cfg, cfg.sparsities[0], PEN, heads=[0, 55],
+                     blocks=[0, 31, 32, 33, 34, 100, 500, 928, 929, 930, 1500, 1825, 1826])
+
+
+# ---------------------------------------------------------- failure paths
+
+def test_bounded_wait_reports_timeout():
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    h3.selftest_timeout(ws, 1000)
+    assert h3.check(ws) == h3.ETIMEOUT
+    assert h3.check(ws) == h3.OK          # the status word was cleared
+
+
+def test_corrupt_routed_list_is_flagged_not_used():
+    cfg = inputs.custom(1, 128, _layout(64, 0, 0, 0, 8, 64), seed=3, cluster_norm=2.0)
+    x = make(cfg)
+    p = h3.plan(1, cfg.S, 128, x["seg"], sparsity=0.5)
+    ws = h3.workspace(p)
+    sel = h3.route(p, x["q_d"], x["k_d"], ws)
+    bad = sel.clone()
+    bad[0, 0, 0] = 100000                 # far outside the key blocks
+    bad[0, 1, 1] = 0                      # a forced block is not a video block
+    h3.forward(p, x["q_d"], x["k_d"], x["v_d"], x["seg_d"], x["times_d"], pen=None, kv_sel=bad, ws=ws)
+    assert h3.check(ws) == h3.EDATA
