@@ -216,6 +216,9 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     cfg = inputs.CONFIGS[CONFIG_ID]
+    if args.heads is not None:
+        cfg = inputs.custom(args.heads, cfg.d, cfg.segments, cfg.seed, cluster_norm=cfg.cluster_norm,
+                            penalty=cfg.penalty, sparsities=cfg.sparsities, name=f"{cfg.name} ({args.heads} heads)")
     seed = cfg.seed + rank
     seg, times, _ = cfg.layout()
     H, S, d = cfg.H, cfg.S, cfg.d
@@ -302,20 +305,22 @@ def run_ours(args, rank, world, local_rank):
         h3.forward(p, qd, kd, vd, seg_d, times_d, pen=pen, kv_sel=sel, ws=ws, out=o)
         o_h.copy_(o.view(torch.int16).view(-1), non_blocking=True)
 
-    e2e_step()
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
+    e2e_ms = float("nan")
+    if not args.no_e2e:
         e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    if h3.check(ws) != h3.OK:
-        raise RuntimeError("device status after e2e")
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = e0.elapsed_time(e1)
+        if h3.check(ws) != h3.OK:
+            raise RuntimeError("device status after e2e")
 
     # max over ranks
     t = torch.tensor([ms, e2e_ms, fwd_ms, route_ms], dtype=torch.float64, device=dev)
@@ -354,6 +359,10 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms / args.steps},
     }
+    if args.no_e2e:
+        line["e2e"] = None
+    if args.heads is not None:
+        line["config"]["workload"] = WORKLOAD.replace("H=56", f"H={args.heads}") + " (profiling variant)"
     if not args.no_cpu_baseline and world == 1:
         small = inputs.custom(1, d, cfg.segments, seed, cluster_norm=cfg.cluster_norm)
         qs, ks, vs = (inputs.tensor(small, i) for i in range(3))
@@ -372,6 +381,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--heads", type=int, default=None,
+                    help="run the same packing with fewer heads (profiling captures only; the default is 56)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
