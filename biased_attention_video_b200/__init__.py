@@ -23,7 +23,8 @@ OK, EINVAL, EUNSUPPORTED, EALIGN, ECUDA, ETIMEOUT, EWORKSPACE, EDATA = 0, -1, -2
 SEG_TEXT, SEG_IMAGE_REF, SEG_AUDIO, SEG_GUIDE, SEG_OUTPUT = 0, 1, 2, 3, 4
 
 # every symbol the C header declares
-EXPORTS = ("h3attn_plan_init", "h3attn_workspace_bytes", "h3attn_pool", "h3attn_route", "h3attn_forward",
+EXPORTS = ("h3attn_plan_init", "h3attn_workspace_bytes", "h3attn_pool", "h3attn_route", "h3attn_route_static",
+           "h3attn_forward",
            "h3attn_dense_workspace_bytes", "h3attn_dense_biased", "h3attn_check", "h3attn_selftest_timeout",
            "h3attn_strerror")
 
@@ -74,6 +75,8 @@ def lib():
         L.h3attn_pool.restype = ctypes.c_int
         L.h3attn_route.argtypes = [PP, _P, _P, _P, _P, ctypes.c_size_t, _P]
         L.h3attn_route.restype = ctypes.c_int
+        L.h3attn_route_static.argtypes = [PP, _P, _P, _P, _P]
+        L.h3attn_route_static.restype = ctypes.c_int
         L.h3attn_forward.argtypes = [PP, _P, _P, _P, _P, _P, ctypes.POINTER(Penalty), _P, _P, _P, _P,
                                      ctypes.c_size_t, _P]
         L.h3attn_forward.restype = ctypes.c_int
@@ -161,6 +164,18 @@ def route(p: Plan, q: torch.Tensor, k: torch.Tensor, ws: torch.Tensor, kv_sel=No
         kv_sel = torch.empty((p.H, p.n_video_blocks, p.k), dtype=torch.int32, device=q.device)
     _raise(lib().h3attn_route(ctypes.byref(p), q.data_ptr(), k.data_ptr(), kv_sel.data_ptr(), ws.data_ptr(),
                               ws.numel(), _stream(stream)), "route")
+    return kv_sel
+
+
+def route_static(p: Plan, q: torch.Tensor, k: torch.Tensor, kv_sel=None, stream=None) -> torch.Tensor:
+    """Same result as route(), for callers that cannot allocate device memory: the
+    pooled centroids live in a fixed 32 MiB array inside the library (no workspace).
+    The output buffer kv_sel may be passed in; concurrent calls share that array."""
+    _check_qkv(q, k)
+    if kv_sel is None:
+        kv_sel = torch.empty((p.H, p.n_video_blocks, p.k), dtype=torch.int32, device=q.device)
+    _raise(lib().h3attn_route_static(ctypes.byref(p), q.data_ptr(), k.data_ptr(), kv_sel.data_ptr(),
+                                     _stream(stream)), "route_static")
     return kv_sel
 
 

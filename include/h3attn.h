@@ -138,6 +138,23 @@ H3ATTN_API int h3attn_pool(const h3attn_plan* plan, const uint16_t* x, int first
 H3ATTN_API int h3attn_route(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, int32_t* kv_sel,
                  void* ws, size_t ws_bytes, void* stream);
 
+/* Routing with no workspace and no allocation.  The pages have no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory when they route (a framework that owns all device memory
+ * through its own pool, a loop that must not pay cudaMalloc's implicit
+ * synchronisation, a host with a fixed memory budget).
+ * Same result as h3attn_route.  Its scratch for the pooled Q and K is a fixed
+ * 32 MiB array inside the library that every GPU loading the library holds
+ * until the process exits; problems with 2 * H * n_video_blocks * d > 8,388,608
+ * are rejected with H3ATTN_EWORKSPACE.  Every call overwrites all the scratch
+ * it reads, so nothing needs clearing between calls; calls that overlap on the
+ * GPU (other streams, other threads) share the array and race.  The first call
+ * on a device looks up the array's device address with that device current;
+ * make that first call before any stream capture.  Allocates nothing and calls
+ * no allocating routine. */
+H3ATTN_API int h3attn_route_static(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, int32_t* kv_sel,
+                                   void* stream);
+
 /* Exact attention over the routed tiles with the temporal penalty.
  * Each query row attends: all keys if its block is a forced (non-video)
  * block or kv_sel is NULL; otherwise the forced key blocks plus the routed

@@ -1,0 +1,50 @@
+"""h3attn_route_static: routing for callers that cannot allocate device memory.
+
+Such a caller (a framework that owns all device memory through its own pool, a
+loop that must not pay cudaMalloc's implicit synchronisation, a host with a
+fixed memory budget) cannot hand over a workspace, so this entry point keeps
+its pooled-centroid scratch in a fixed array inside the library.  These tests
+call it through the C ABI and check it returns exactly what h3attn_route
+returns, on two different calls in a row (the second call must not see the
+first call's scratch contents)."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import biased_attention_video_b200 as h3
+import inputs
+from parity import make
+
+
+def _route_static_abi(p, q, k):
+    sel = torch.full((p.H, p.n_video_blocks, p.k), -1, dtype=torch.int32, device=q.device)
+    rc = h3.lib().h3attn_route_static(ctypes.byref(p), q.data_ptr(), k.data_ptr(), sel.data_ptr(),
+                                      torch.cuda.current_stream().cuda_stream)
+    assert rc == h3.OK, h3.lib().h3attn_strerror(rc)
+    return sel
+
+
+@pytest.mark.gpu
+def test_route_static_matches_route_on_consecutive_calls():
+    cfg2 = inputs.CONFIGS[2]
+    c3 = inputs.CONFIGS[3]
+    cfg3 = inputs.custom(8, c3.d, c3.segments, c3.seed, cluster_norm=c3.cluster_norm)
+    for cfg, s in [(cfg2, 0.85), (cfg3, 0.60)]:
+        x = make(cfg)
+        p = h3.plan(cfg.H, cfg.S, cfg.d, x["seg"], sparsity=s)
+        static_sel = _route_static_abi(p, x["q_d"], x["k_d"])
+        ws = h3.workspace(p)
+        ref = h3.route(p, x["q_d"], x["k_d"], ws)
+        torch.cuda.synchronize()
+        assert h3.check(ws) == h3.OK
+        assert torch.equal(static_sel, ref), cfg.name
+
+
+def test_route_static_rejects_problems_beyond_its_scratch():
+    """Checked on the host before any device work: 56 heads x 1794 video blocks x d=128 is too large."""
+    seg, _, _ = inputs.CONFIGS[5].layout()
+    p = h3.plan(56, 116883, 128, seg, sparsity=0.9)
+    fake = 1 << 40
+    assert h3.lib().h3attn_route_static(ctypes.byref(p), fake, fake, fake, None) == h3.EWORKSPACE
