@@ -127,8 +127,6 @@ int forward_impl(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, 
   p.wait_polls = kWaitPolls;
   p.wait_ns = kWaitNs;
   const int n_qtiles = (plan->n_blocks + 1) / 2;
-  p.n_dense_tiles = routed ? (plan->first_video_block + 1) / 2 : n_qtiles;
-  if (p.n_dense_tiles > n_qtiles) p.n_dense_tiles = n_qtiles;
 
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, q, plan->H, plan->S, plan->d) || !make_map(&tk, k, plan->H, plan->S, plan->d) ||

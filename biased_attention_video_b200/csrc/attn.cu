@@ -10,16 +10,23 @@
 // lists in 128-key tiles (two 64-row key blocks per tile); each query row
 // masks the key blocks its own query block does not attend.
 //
-// Warp roles (256 threads):
-//   warp 0      TMA producer: Q tile once, then K and V tiles into a 2-stage ring
+// Two CTAs share an SM (TMEM 256 columns and < 113 KB of shared memory each),
+// so one CTA's tensor-core work overlaps the other's softmax.
+//
+// Warp roles (192 threads; two CTAs per SM leave 168 registers per thread):
+//   warp 0      TMA producer: Q tile once, then K and V 128-key tiles
 //   warp 1      TMEM owner + single-thread tcgen05.mma issuer
-//   warps 4..7  softmax: thread = one query row = one TMEM lane
-// TMEM (512 columns): S0 [0,128), S1 [128,256) double-buffered scores, the
-// bf16 probabilities P(j) written over the first 64 columns of S(j & 1),
-// O [256, 256 + d).
-// MMA issue order S(0), S(1), PV(0), S(2), PV(1), ...: tcgen05.mma ops of one
-// thread run in issue order, so S(j) never overwrites P(j-2) before PV(j-2)
-// has read it, and the commit after S(j) also covers PV(j-2).
+//   warps 2..5  softmax: thread = one query row = one TMEM lane; warp w may
+//               only touch TMEM lanes [32 (w % 4), 32 (w % 4) + 32)
+// TMEM: S [0,128) fp32 scores; the bf16 probabilities P(j) are written over
+// its first 64 columns; O [128, 128 + d).
+// The softmax works on one 64-key half of a tile at a time (64 live scores per
+// thread, so the kernel fits the 128 registers two CTAs per SM allow) and
+// hands over P half by half; the MMA warp issues PV(j, half 0) while the
+// softmax works on half 1.
+// MMA issue order S(0), PV(0,0), PV(0,1), S(1), ...: the tcgen05.mma ops of one
+// thread run in issue order, so S(j+1) never overwrites P(j) before PV(j) has
+// read it, and when the commit after S(j+1) fires, PV(j) is complete too.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -30,12 +37,14 @@
 namespace h3 {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kStages = 2;
+constexpr int kThreads = 192;
 constexpr int kTileRows = 128;  // query rows per CTA
 constexpr int kTileKeys = 128;  // keys per KV tile
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemO = 128;  // O column offset
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
+constexpr unsigned kFull = 0xFFFFFFFFu;
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -52,50 +61,32 @@ __device__ __forceinline__ void report(int* status, int code) { atomicCAS(status
 
 template <int D>
 struct Layout {
-  static constexpr int kHalves = D / 64;                 // 128-byte swizzle atoms along d
-  static constexpr int kHalfBytes = kTileRows * 128;     // one d-half of a 128-row tile
+  static constexpr int kHalves = D / 64;               // 128-byte swizzle atoms along d
+  static constexpr int kHalfBytes = kTileRows * 128;   // one d-half of a 128-row tile
   static constexpr int kTileBytes = kHalves * kHalfBytes;
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kTileBytes;
-  static constexpr int kV = kK + kStages * kTileBytes;
-  static constexpr int kBars = kV + kStages * kTileBytes;
-  // barriers: q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_full[2], o_done, o_final, drain
-  static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 3;
-  static constexpr int kMisc = kBars + kNumBars * 8;      // tmem base, abort, n_entries
+  static constexpr int kV = kK + kTileBytes;
+  static constexpr int kBars = kV + kTileBytes;
+  // barriers: q_full, k_full, k_empty, v_full, v_empty, s_full, p_full[2], o_half0, o_final, drain
+  static constexpr int kNumBars = 11;
+  static constexpr int kMisc = kBars + kNumBars * 8;  // tmem base, abort flag, n_entries
   static constexpr int kBitmaps = kMisc + 16;
   static int host_bytes(int n_blocks) {
-    int nwords = (n_blocks + 31) / 32;
-    return 1024 /*alignment slack*/ + kBitmaps + 2 * nwords * 4 + n_blocks * 4;
+    const int nwords = (n_blocks + 31) / 32;
+    return 1024 /*alignment slack*/ + kBitmaps + 2 * nwords * 4 + ((n_blocks * 2 + 15) & ~15);
   }
 };
 
 struct Bars {
-  uint64_t* q_full;
-  uint64_t* k_full;
-  uint64_t* k_empty;
-  uint64_t* v_full;
-  uint64_t* v_empty;
-  uint64_t* s_full;
-  uint64_t* p_full;
-  uint64_t* o_done;
-  uint64_t* o_final;
-  uint64_t* drain;
+  uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *o_half0, *o_final, *drain;
 };
 
+// p_full[h]: P of half h of the current tile is in TMEM (one completion per
+// tile each, so a waiter is never more than one phase behind).
 __device__ __forceinline__ Bars carve_bars(uint8_t* base) {
   uint64_t* b = reinterpret_cast<uint64_t*>(base);
-  Bars r;
-  r.q_full = b;
-  r.k_full = b + 1;
-  r.k_empty = b + 1 + kStages;
-  r.v_full = b + 1 + 2 * kStages;
-  r.v_empty = b + 1 + 3 * kStages;
-  r.s_full = b + 1 + 4 * kStages;
-  r.p_full = b + 3 + 4 * kStages;
-  r.o_done = b + 5 + 4 * kStages;
-  r.o_final = b + 6 + 4 * kStages;
-  r.drain = b + 7 + 4 * kStages;
-  return r;
+  return Bars{b, b + 1, b + 2, b + 3, b + 4, b + 5, b + 6, b + 8, b + 9, b + 10};
 }
 
 // Bounded wait with CTA-wide abort.  On give-up: raise the CTA abort flag and
@@ -137,56 +128,57 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, const
   }
 }
 
+__device__ __forceinline__ float block_penalty_log2(float tq, float tk, const AttnParams& p) {
+  const float dt = fabsf(tq - tk);
+  const float ex = fmaxf(dt - p.window, 0.0f) * p.inv_falloff;
+  return fminf(p.strength_log2 * ex * ex, p.cap_log2);
+}
+
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using L = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Bars bars = carve_bars(smem + L::kBars);
+  const Bars bars = carve_bars(smem + L::kBars);
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   int* n_entries_slot = reinterpret_cast<int*>(smem + L::kMisc + 8);
   const int nwords = (p.n_blocks + 31) >> 5;
   uint32_t* bm_a = reinterpret_cast<uint32_t*>(smem + L::kBitmaps);
   uint32_t* bm_b = bm_a + nwords;
-  uint32_t* list = bm_b + nwords;
+  // entry = key block (14 bits) | attended by block A << 14 | attended by block B << 15
+  uint16_t* list = reinterpret_cast<uint16_t*>(bm_b + nwords);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // Tile order: heaviest (dense) query tiles first, head-minor inside a class.
-  int head, qtile;
-  {
-    const int lin = blockIdx.x;
-    const int heavy = p.n_dense_tiles * p.H;
-    if (lin < heavy) {
-      head = lin % p.H;
-      qtile = lin / p.H;
-    } else {
-      const int r = lin - heavy;
-      head = r % p.H;
-      qtile = p.n_dense_tiles + r / p.H;
-    }
-  }
-  if (*reinterpret_cast<volatile int*>(p.status) == kStatusTimeout) return;  // an earlier CTA gave up
+  // Tile order: head-major, so the ~300 CTAs resident at a time share one or
+  // two heads' K/V in L2; inside a head the dense (prefix) query tiles come
+  // first, so the longest tiles start earliest.
+  const int n_qtiles = (p.n_blocks + 1) >> 1;
+  const int head = (int)(blockIdx.x / n_qtiles);
+  const int qtile = (int)(blockIdx.x % n_qtiles);
+  // An earlier CTA that gave up leaves the status word set: skip the work
+  // (decided once per CTA so that every thread leaves together).
+  if (tid == 0) *abort_flag = *reinterpret_cast<volatile int*>(p.status) == kStatusTimeout ? 1 : 0;
+  __syncthreads();
+  if (*abort_flag) return;
+  __syncthreads();
 
   if (tid == 0) {
     *abort_flag = 0;
     mbar_init(bars.q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(bars.k_full + s, 1);
-      mbar_init(bars.k_empty + s, 1);
-      mbar_init(bars.v_full + s, 1);
-      mbar_init(bars.v_empty + s, 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bars.s_full + b, 1);
-      mbar_init(bars.p_full + b, 128);
-    }
-    mbar_init(bars.o_done, 1);
+    mbar_init(bars.k_full, 1);
+    mbar_init(bars.k_empty, 1);
+    mbar_init(bars.v_full, 1);
+    mbar_init(bars.v_empty, 1);
+    mbar_init(bars.s_full, 1);
+    mbar_init(bars.p_full, 128);
+    mbar_init(bars.p_full + 1, 128);
+    mbar_init(bars.o_half0, 1);
     mbar_init(bars.o_final, 1);
     mbar_init(bars.drain, 1);
     fence_mbar_init();
@@ -195,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_v);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_base_slot, 512);
+    tmem_alloc(tmem_base_slot, kTmemCols);
     tmem_relinquish();
   }
 
@@ -206,48 +198,48 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool dense_b = p.kv_sel == nullptr || qb_b < p.first_video_block;
   for (int w = tid; w < nwords; w += kThreads) {
     const int lo = w * 32;
-    uint32_t full = (p.n_blocks - lo >= 32) ? 0xFFFFFFFFu : ((1u << (p.n_blocks - lo)) - 1u);
-    int nf = p.first_video_block - lo;
-    uint32_t forced = nf <= 0 ? 0u : (nf >= 32 ? 0xFFFFFFFFu : ((1u << nf) - 1u));
+    const uint32_t full = (p.n_blocks - lo >= 32) ? 0xFFFFFFFFu : ((1u << (p.n_blocks - lo)) - 1u);
+    const int nf = p.first_video_block - lo;
+    const uint32_t forced = nf <= 0 ? 0u : (nf >= 32 ? 0xFFFFFFFFu : ((1u << nf) - 1u));
     bm_a[w] = !has_a ? 0u : (dense_a ? full : forced);
     bm_b[w] = !has_b ? 0u : (dense_b ? full : forced);
   }
   __syncthreads();
-  if (has_a && !dense_a) {
-    const int32_t* lst = p.kv_sel + ((size_t)head * p.n_video_blocks + (qb_a - p.first_video_block)) * p.k;
-    for (int i = tid; i < p.k; i += kThreads) {
-      int e = lst[i];
-      if (e < p.first_video_block || e >= p.n_blocks) report(p.status, kStatusData);
-      else atomicOr(bm_a + (e >> 5), 1u << (e & 31));
-    }
-  }
-  if (has_b && !dense_b) {
-    const int32_t* lst = p.kv_sel + ((size_t)head * p.n_video_blocks + (qb_b - p.first_video_block)) * p.k;
-    for (int i = tid; i < p.k; i += kThreads) {
-      int e = lst[i];
-      if (e < p.first_video_block || e >= p.n_blocks) report(p.status, kStatusData);
-      else atomicOr(bm_b + (e >> 5), 1u << (e & 31));
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int qb = half == 0 ? qb_a : qb_b;
+    const bool routed = half == 0 ? (has_a && !dense_a) : (has_b && !dense_b);
+    uint32_t* bm = half == 0 ? bm_a : bm_b;
+    if (routed) {
+      const int32_t* lst = p.kv_sel + ((size_t)head * p.n_video_blocks + (qb - p.first_video_block)) * p.k;
+      for (int i = tid; i < p.k; i += kThreads) {
+        const int e = lst[i];
+        if (e < p.first_video_block || e >= p.n_blocks) report(p.status, kStatusData);
+        else atomicOr(bm + (e >> 5), 1u << (e & 31));
+      }
     }
   }
   __syncthreads();
   if (warp == 0) {
     // lane l owns words [l*per, (l+1)*per)
     const int per = (nwords + 31) / 32;
+    const int w0 = lane * per, w1 = min(nwords, (lane + 1) * per);
     int cnt = 0;
-    for (int w = lane * per; w < min(nwords, (lane + 1) * per); ++w) cnt += __popc(bm_a[w] | bm_b[w]);
+    for (int w = w0; w < w1; ++w) cnt += __popc(bm_a[w] | bm_b[w]);
     int incl = cnt;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      const int v = __shfl_up_sync(kFull, incl, o);
       if (lane >= o) incl += v;
     }
     int pos = incl - cnt;
-    for (int w = lane * per; w < min(nwords, (lane + 1) * per); ++w) {
-      uint32_t a = bm_a[w], b = bm_b[w], u = a | b;
+    for (int w = w0; w < w1; ++w) {
+      const uint32_t a = bm_a[w], b = bm_b[w];
+      uint32_t u = a | b;
       while (u) {
         const int bit = __ffs(u) - 1;
         u &= u - 1;
-        list[pos++] = (uint32_t)(w * 32 + bit) | (((a >> bit) & 1u) << 16) | (((b >> bit) & 1u) << 17);
+        list[pos++] = (uint16_t)((w * 32 + bit) | (((a >> bit) & 1u) << 14) | (((b >> bit) & 1u) << 15));
       }
     }
     if (lane == 31) *n_entries_slot = incl;
@@ -259,12 +251,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_entries = *n_entries_slot;
   const int n_tiles = (n_entries + 1) >> 1;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      uint32_t issued_k[kStages] = {0, 0}, issued_v[kStages] = {0, 0};
+  if (warp < 2) {
+    if (warp == 0 && lane == 0) {
+      // ---------------------------------------------------------- producer
+      uint32_t issued_k = 0, issued_v = 0;
       const int q_row0 = qtile * kTileRows;
       uint8_t* sq = smem + L::kQ;
+      uint8_t* sk = smem + L::kK;
+      uint8_t* sv = smem + L::kV;
       mbar_arrive_expect_tx(bars.q_full, L::kTileBytes);
 #pragma unroll
       for (int c = 0; c < L::kHalves; ++c) {
@@ -273,99 +267,94 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int oob_row = p.n_blocks * 64;  // a whole block past S: zero-filled by TMA
       for (int j = 0; j < n_tiles; ++j) {
-        const int s = j % kStages;
-        const uint32_t ph = (uint32_t)(j / kStages) & 1u;
-        const int e0 = (int)(list[2 * j] & 0xFFFFu);
-        const int e1 = (2 * j + 1 < n_entries) ? (int)(list[2 * j + 1] & 0xFFFFu) : -1;
+        const uint32_t ph = (uint32_t)j & 1u;
+        const int e0 = (int)(list[2 * j] & 0x3FFFu);
+        const int e1 = (2 * j + 1 < n_entries) ? (int)(list[2 * j + 1] & 0x3FFFu) : -1;
         const int r0 = e0 * 64, r1 = e1 >= 0 ? e1 * 64 : oob_row;
-        if (!wait_bar(bars.k_empty + s, ph ^ 1u, p, abort_flag)) break;
-        uint8_t* sk = smem + L::kK + s * L::kTileBytes;
-        mbar_arrive_expect_tx(bars.k_full + s, L::kTileBytes);
+        if (!wait_bar(bars.k_empty, ph ^ 1u, p, abort_flag)) break;
+        mbar_arrive_expect_tx(bars.k_full, L::kTileBytes);
 #pragma unroll
         for (int c = 0; c < L::kHalves; ++c) {
-          tma_load_3d(sk + c * L::kHalfBytes, &tm_k, bars.k_full + s, c * 64, r0, head);
-          tma_load_3d(sk + c * L::kHalfBytes + 8192, &tm_k, bars.k_full + s, c * 64, r1, head);
+          tma_load_3d(sk + c * L::kHalfBytes, &tm_k, bars.k_full, c * 64, r0, head);
+          tma_load_3d(sk + c * L::kHalfBytes + 8192, &tm_k, bars.k_full, c * 64, r1, head);
         }
-        ++issued_k[s];
-        if (!wait_bar(bars.v_empty + s, ph ^ 1u, p, abort_flag)) break;
-        uint8_t* sv = smem + L::kV + s * L::kTileBytes;
-        mbar_arrive_expect_tx(bars.v_full + s, L::kTileBytes);
+        ++issued_k;
+        if (!wait_bar(bars.v_empty, ph ^ 1u, p, abort_flag)) break;
+        mbar_arrive_expect_tx(bars.v_full, L::kTileBytes);
 #pragma unroll
         for (int c = 0; c < L::kHalves; ++c) {
-          tma_load_3d(sv + c * L::kHalfBytes, &tm_v, bars.v_full + s, c * 64, r0, head);
-          tma_load_3d(sv + c * L::kHalfBytes + 8192, &tm_v, bars.v_full + s, c * 64, r1, head);
+          tma_load_3d(sv + c * L::kHalfBytes, &tm_v, bars.v_full, c * 64, r0, head);
+          tma_load_3d(sv + c * L::kHalfBytes + 8192, &tm_v, bars.v_full, c * 64, r1, head);
         }
-        ++issued_v[s];
+        ++issued_v;
       }
       // drain: every issued load must land before the CTA may exit
       drain_wait(bars.q_full, 0, p);
-      for (int s = 0; s < kStages; ++s) {
-        if (issued_k[s]) drain_wait(bars.k_full + s, (issued_k[s] - 1) & 1u, p);
-        if (issued_v[s]) drain_wait(bars.v_full + s, (issued_v[s] - 1) & 1u, p);
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+      if (issued_k) drain_wait(bars.k_full, (issued_k - 1) & 1u, p);
+      if (issued_v) drain_wait(bars.v_full, (issued_v - 1) & 1u, p);
+    } else if (warp == 1 && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t kIdescS = idesc_bf16_f32(128, kTileKeys, 0, 0);
       constexpr uint32_t kIdescO = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t q_addr = smem_u32(smem + L::kQ);
-      const uint32_t tmem_o = tmem_base + 256;
-      bool ok = wait_bar(bars.q_full, 0, p, abort_flag);
-      auto issue_pv = [&](int jj) -> bool {
-        const int s = jj % kStages;
-        const uint32_t ph = (uint32_t)(jj / kStages) & 1u;
-        if (!wait_bar(bars.p_full + (jj & 1), (uint32_t)(jj >> 1) & 1u, p, abort_flag)) return false;
-        if (!wait_bar(bars.v_full + s, ph, p, abort_flag)) return false;
+      const uint32_t k_addr = smem_u32(smem + L::kK);
+      const uint32_t v_addr = smem_u32(smem + L::kV);
+      const uint32_t tmem_s = tmem_base;
+      const uint32_t tmem_o = tmem_base + kTmemO;
+      auto issue_s = [&](int j) -> bool {
+        if (!wait_bar(bars.k_full, (uint32_t)j & 1u, p, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t v_addr = smem_u32(smem + L::kV + s * L::kTileBytes);
-        const uint32_t p_tmem = tmem_base + (uint32_t)(jj & 1) * 128;
-#pragma unroll
-        for (int kk = 0; kk < kTileKeys / 16; ++kk) {
-          // B = V tile, MN-major: 16 keys per step = two 8-row swizzle groups
-          const uint64_t bdesc = sw128_desc(v_addr + kk * 2048, L::kHalfBytes, 1024);
-          umma_ts(tmem_o, p_tmem + kk * 8, bdesc, kIdescO, (jj > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(bars.o_done);
-        umma_commit(bars.v_empty + s);
-        return true;
-      };
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        const int s = j % kStages;
-        const uint32_t ph = (uint32_t)(j / kStages) & 1u;
-        if (!wait_bar(bars.k_full + s, ph, p, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(smem + L::kK + s * L::kTileBytes);
-        const uint32_t s_tmem = tmem_base + (uint32_t)(j & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int c = kk >> 2, off = (kk & 3) * 32;
           const uint64_t adesc = sw128_desc(q_addr + c * L::kHalfBytes + off, 16, 1024);
           const uint64_t bdesc = sw128_desc(k_addr + c * L::kHalfBytes + off, 16, 1024);
-          umma_ss(s_tmem, adesc, bdesc, kIdescS, kk > 0 ? 1u : 0u);
+          umma_ss(tmem_s, adesc, bdesc, kIdescS, kk > 0 ? 1u : 0u);
         }
-        umma_commit(bars.s_full + (j & 1));
-        umma_commit(bars.k_empty + s);
-        if (j >= 1 && !issue_pv(j - 1)) {
+        umma_commit(bars.s_full);
+        umma_commit(bars.k_empty);
+        return true;
+      };
+      bool ok = wait_bar(bars.q_full, 0, p, abort_flag);
+      if (ok && n_tiles > 0) ok = issue_s(0);
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const uint32_t ph = (uint32_t)j & 1u;
+        if (!wait_bar(bars.v_full, ph, p, abort_flag)) {
           ok = false;
           break;
         }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          if (!wait_bar(bars.p_full + hh, ph, p, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = hh * 4; kk < hh * 4 + 4; ++kk) {
+            // B = V tile, MN-major: 16 keys per step = two 8-row swizzle groups
+            const uint64_t bdesc = sw128_desc(v_addr + kk * 2048, L::kHalfBytes, 1024);
+            umma_ts(tmem_o, tmem_s + kk * 8, bdesc, kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(hh == 0 ? bars.o_half0 : bars.v_empty);
+        }
+        if (ok && j + 1 < n_tiles) ok = issue_s(j + 1);
       }
-      if (ok && n_tiles > 0) ok = issue_pv(n_tiles - 1);
       umma_commit(bars.o_final);
       // drain: all issued MMAs complete before TMEM is released
       umma_commit(bars.drain);
       drain_wait(bars.drain, 0, p);
     }
-  } else if (warp >= 4) {
+  } else {
     // ------------------------------------------------------------ softmax
-    const int r = tid - 128;  // row within the tile == TMEM lane
+    // tcgen05.ld/st are warp-collective (.sync.aligned): every branch that
+    // guards one is made warp-uniform with __all_sync / __any_sync.
     const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // row within the tile == TMEM lane
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-    const int my_half = r >> 6;  // 0: query block A, 1: query block B
+    const uint32_t t_s = tmem_base + lane_addr;
+    const uint32_t t_o = tmem_base + lane_addr + kTmemO;
+    const int my_bit = 14 + (r >> 6);  // list bit of this row's query block
     const int qrow = qtile * kTileRows + r;
     const bool row_valid = qrow < p.S;
     const bool pen_row = p.pen_on && row_valid && p.seg[qrow] == kSegOutput;
@@ -374,142 +363,138 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m = -INFINITY;  // running max, log2 units (upper bound of the true max)
     float l = 0.0f;
     bool ok = true;
-    // tcgen05.ld/st are warp-collective (.sync.aligned): every branch that
-    // guards one is made warp-uniform with __all_sync / __any_sync.
-    constexpr unsigned kFull = 0xFFFFFFFFu;
-    for (int j = 0; j < n_tiles; ++j) {
-      const int buf = j & 1;
-      const bool got = wait_bar(bars.s_full + buf, (uint32_t)(j >> 1) & 1u, p, abort_flag);
+    for (int j = 0; ok && j < n_tiles; ++j) {
+      const bool got = wait_bar(bars.s_full, (uint32_t)j & 1u, p, abort_flag);
       if (!__all_sync(kFull, got)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float sv[kTileKeys];
-      {
-        uint32_t tmp[32];
 #pragma unroll
-        for (int c = 0; c < kTileKeys / 32; ++c) {
+      for (int hh = 0; hh < 2; ++hh) {
+        // this half: 0 skip, 1 plain, 2 constant penalty, 3 per-key penalty
+        int mode = 0, nv = 0, kblock = 0;
+        float cpen = 0.0f;
+        const int idx = 2 * j + hh;
+        if (idx < n_entries) {
+          const uint32_t ent = list[idx];
+          kblock = (int)(ent & 0x3FFFu);
+          if ((ent >> my_bit) & 1u) {
+            const uint2 kd = p.kv_desc[kblock];
+            nv = (int)(kd.x & 0xFFu);
+            const int kind = (int)((kd.x >> 8) & 3u);
+            mode = 1;
+            if (pen_row && kind == 1) {
+              cpen = block_penalty_log2(tq, __uint_as_float(kd.y), p);
+              mode = 2;
+            } else if (pen_row && kind == 2) {
+              mode = 3;
+            }
+          }
+        }
+        float sv[64];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t tmp[32];
           __syncwarp();
-          tmem_ld32(tmem_base + lane_addr + (uint32_t)buf * 128 + c * 32, tmp);
+          tmem_ld32(t_s + hh * 64 + c * 32, tmp);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(tmp[i]);
         }
-      }
-      // per 64-key half: attended? penalty mode? valid keys?
-      int mode[2];      // 0 skip, 1 plain, 2 constant penalty, 3 per-key penalty
-      int nvalid[2];
-      float cpen[2];
-      int kblock[2];
+        float mx = -INFINITY;
+        if (mode != 0) {
+          if (nv == 64) {
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int idx = 2 * j + hh;
-        mode[hh] = 0;
-        nvalid[hh] = 0;
-        cpen[hh] = 0.0f;
-        kblock[hh] = 0;
-        if (idx < n_entries) {
-          const uint32_t ent = list[idx];
-          const bool att = ((ent >> (16 + my_half)) & 1u) != 0;
-          const int b = (int)(ent & 0xFFFFu);
-          kblock[hh] = b;
-          if (att) {
-            const uint2 kd = p.kv_desc[b];
-            nvalid[hh] = (int)(kd.x & 0xFFu);
-            const int kind = (int)((kd.x >> 8) & 3u);
-            mode[hh] = 1;
-            if (pen_row && kind == 1) {
-              const float dt = fabsf(tq - __uint_as_float(kd.y));
-              const float ex = fmaxf(dt - p.window, 0.0f) * p.inv_falloff;
-              cpen[hh] = fminf(p.strength_log2 * ex * ex, p.cap_log2);
-              mode[hh] = 2;
-            } else if (pen_row && kind == 2) {
-              mode[hh] = 3;
-            }
+            for (int i = 0; i < 64; ++i) mx = fmaxf(mx, sv[i]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 64; ++i)
+              if (i < nv) mx = fmaxf(mx, sv[i]);
           }
         }
-      }
-      float mx = -INFINITY;
+        mx *= scale;
+        // Conditional rescale: the running max only moves when it grows by
+        // more than 2^8; below that the stale max keeps every probability <= 256.
+        const bool grow = mx > m + kRescaleThreshold;
+        const bool o_rescale = grow && l > 0.0f;
+        float alpha = 1.0f;
+        if (__any_sync(kFull, o_rescale)) {
+          // Half 0: O is stable (PV(j-1) completed before S(j) did).  Half 1:
+          // wait for PV(j, half 0), issued once P of half 0 was handed over.
+          if (hh == 1) {
+            const bool got2 = wait_bar(bars.o_half0, (uint32_t)j & 1u, p, abort_flag);
+            if (!__all_sync(kFull, got2)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          alpha = o_rescale ? ex2(m - mx) : 1.0f;
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        if (mode[hh] == 0) continue;
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t tmp[32];
+            __syncwarp();
+            tmem_ld32(t_o + c * 32, tmp);
+            tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if (i < nvalid[hh]) mx = fmaxf(mx, sv[hh * 64 + i]);
-      }
-      mx *= scale;
-      // Conditional rescale: the running max only moves when it grows by more
-      // than 2^8; below that the stale max keeps every probability <= 256.
-      const bool grow = mx > m + kRescaleThreshold;
-      const bool o_rescale = grow && l > 0.0f;
-      if (__any_sync(kFull, o_rescale)) {
-        // O holds PV(0..j-1): wait for PV(j-1), then scale it in place
-        // (lanes that do not rescale multiply by 1).
-        const bool got2 = wait_bar(bars.o_done, (uint32_t)(j - 1) & 1u, p, abort_flag);
-        if (!__all_sync(kFull, got2)) {
-          ok = false;
-          break;
+            for (int i = 0; i < 32; ++i) tmp[i] = __float_as_uint(__uint_as_float(tmp[i]) * alpha);
+            tmem_st32(t_o + c * 32, tmp);
+          }
         }
-        tc_fence_after();
-        const float alpha = o_rescale ? ex2(m - mx) : 1.0f;
-        uint32_t tmp[32];
+        if (grow) m = mx;
+        // probabilities -> bf16 pairs into columns [32 hh, 32 hh + 32) of S
+        float lt = 0.0f;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          const uint32_t a = tmem_base + lane_addr + 256 + c * 32;
+        for (int c = 0; c < 2; ++c) {
+          uint32_t packed[16];
+          if (mode == 0) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) packed[i] = 0u;
+          } else if (mode == 3) {
+            const int key0 = kblock * 64 + c * 32;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float pp[2];
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int col = c * 32 + 2 * i + e;
+                float pen_k = 0.0f;
+                if (col < nv && p.seg[key0 + 2 * i + e] == kSegGuide)
+                  pen_k = block_penalty_log2(tq, p.times[key0 + 2 * i + e], p);
+                pp[e] = col < nv ? ex2(fmaf(sv[col], scale, -(m + pen_k))) : 0.0f;
+              }
+              lt += pp[0] + pp[1];
+              packed[i] = pack_bf16(pp[0], pp[1]);
+            }
+          } else if (nv == 64) {
+            const float off = -(m + cpen);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float p0 = ex2(fmaf(sv[c * 32 + 2 * i], scale, off));
+              const float p1 = ex2(fmaf(sv[c * 32 + 2 * i + 1], scale, off));
+              lt += p0 + p1;
+              packed[i] = pack_bf16(p0, p1);
+            }
+          } else {
+            const float off = -(m + cpen);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int col = c * 32 + 2 * i;
+              const float p0 = col < nv ? ex2(fmaf(sv[col], scale, off)) : 0.0f;
+              const float p1 = col + 1 < nv ? ex2(fmaf(sv[col + 1], scale, off)) : 0.0f;
+              lt += p0 + p1;
+              packed[i] = pack_bf16(p0, p1);
+            }
+          }
           __syncwarp();
-          tmem_ld32(a, tmp);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) tmp[i] = __float_as_uint(__uint_as_float(tmp[i]) * alpha);
-          tmem_st32(a, tmp);
+          tmem_st16(t_s + hh * 32 + c * 16, packed);
         }
+        l = l * alpha + lt;
         tmem_wait_st();
-        l *= alpha;
+        tc_fence_before();
+        mbar_arrive(bars.p_full + hh);
       }
-      if (grow) m = mx;
-      // probabilities -> bf16 pairs into the first 64 columns of S(buf)
-#pragma unroll
-      for (int c = 0; c < kTileKeys / 32; ++c) {
-        const int hh = c >> 1;
-        uint32_t packed[16];
-        float pr[32];
-        const int md = mode[hh];
-        if (md == 0) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) pr[i] = 0.0f;
-        } else if (md == 3) {
-          const int key0 = kblock[hh] * 64 + (c & 1) * 32;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int col = (c & 1) * 32 + i;
-            float pen_k = 0.0f;
-            if (col < nvalid[hh] && p.seg[key0 + i] == kSegGuide) {
-              const float dt = fabsf(tq - p.times[key0 + i]);
-              const float ex = fmaxf(dt - p.window, 0.0f) * p.inv_falloff;
-              pen_k = fminf(p.strength_log2 * ex * ex, p.cap_log2);
-            }
-            pr[i] = col < nvalid[hh] ? ex2(fmaf(sv[c * 32 + i], scale, -(m + pen_k))) : 0.0f;
-          }
-        } else {
-          const float off = -(m + cpen[hh]);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int col = (c & 1) * 32 + i;
-            pr[i] = col < nvalid[hh] ? ex2(fmaf(sv[c * 32 + i], scale, off)) : 0.0f;
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          l += pr[2 * i] + pr[2 * i + 1];
-          packed[i] = pack_bf16(pr[2 * i], pr[2 * i + 1]);
-        }
-        __syncwarp();
-        tmem_st16(tmem_base + lane_addr + (uint32_t)buf * 128 + c * 16, packed);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bars.p_full + buf);
     }
     // ---------------------------------------------------------- epilogue
     bool fin = __all_sync(kFull, ok) && n_tiles > 0;
@@ -522,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < D / 32; ++c) {
         uint32_t tmp[32];
         __syncwarp();
-        tmem_ld32(tmem_base + lane_addr + 256 + c * 32, tmp);
+        tmem_ld32(t_o + c * 32, tmp);
         tmem_wait_ld();
         uint32_t outw[16];
 #pragma unroll
@@ -531,19 +516,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (row_valid) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(outw[4 * v], outw[4 * v + 1], outw[4 * v + 2], outw[4 * v + 3]);
+          for (int v = 0; v < 4; ++v)
+            dst[v] = make_uint4(outw[4 * v], outw[4 * v + 1], outw[4 * v + 2], outw[4 * v + 3]);
         }
       }
       if (row_valid && p.lse != nullptr) p.lse[(size_t)head * p.S + qrow] = (m + __log2f(l)) * kLn2;
     }
   }
-  // warps 2..3 have no role after the list is built
 
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
+    tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 

@@ -18,7 +18,6 @@ constexpr int kStatusData = 2;
 struct AttnParams {
   int H, S, d;
   int n_blocks, first_video_block, n_video_blocks, k;
-  int n_dense_tiles;           // query tiles holding a dense query block (scheduled first)
   const int32_t* kv_sel;       // [H][nV][k] or null (dense)
   const uint8_t* seg;          // [S]
   const float* times;          // [S]
