@@ -274,6 +274,13 @@ int h3attn_selftest_timeout(void* ws, uint32_t polls, void* stream) {
   return H3ATTN_OK;
 }
 
+int h3attn_selftest_exp2(const float* x, float* y, int n, void* stream) {
+  if (x == nullptr || y == nullptr || n < 0 || (n & 1)) return H3ATTN_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(x) & 7u) || (reinterpret_cast<uintptr_t>(y) & 7u)) return H3ATTN_EALIGN;
+  if (h3::launch_selftest_exp2(x, y, n / 2, static_cast<cudaStream_t>(stream)) != cudaSuccess) return H3ATTN_ECUDA;
+  return H3ATTN_OK;
+}
+
 const char* h3attn_strerror(int status) {
   switch (status) {
     case H3ATTN_OK: return "ok";

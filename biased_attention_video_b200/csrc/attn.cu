@@ -13,17 +13,17 @@
 // Two CTAs share an SM (TMEM 256 columns and < 113 KB of shared memory each),
 // so one CTA's tensor-core work overlaps the other's softmax.
 //
-// Warp roles (192 threads; two CTAs per SM leave 168 registers per thread):
+// Warp roles (320 threads; two CTAs per SM leave 96 registers per thread):
 //   warp 0      TMA producer: Q tile once, then K and V 128-key tiles
 //   warp 1      TMEM owner + single-thread tcgen05.mma issuer
-//   warps 2..5  softmax: thread = one query row = one TMEM lane; warp w may
-//               only touch TMEM lanes [32 (w % 4), 32 (w % 4) + 32)
+//   warps 2..9  softmax: two threads per query row (= TMEM lane), each owning
+//               half of the keys of a tile; warp w may only touch TMEM lanes
+//               [32 (w % 4), 32 (w % 4) + 32)
 // TMEM: S [0,128) fp32 scores; the bf16 probabilities P(j) are written over
 // its first 64 columns; O [128, 128 + d).
-// The softmax works on one 64-key half of a tile at a time (64 live scores per
-// thread, so the kernel fits the 128 registers two CTAs per SM allow) and
-// hands over P half by half; the MMA warp issues PV(j, half 0) while the
-// softmax works on half 1.
+// The softmax works on one 64-key half of a tile at a time and hands over P
+// half by half; the MMA warp issues PV(j, half 0) while the softmax works on
+// half 1.
 // MMA issue order S(0), PV(0,0), PV(0,1), S(1), ...: the tcgen05.mma ops of one
 // thread run in issue order, so S(j+1) never overwrites P(j) before PV(j) has
 // read it, and when the commit after S(j+1) fires, PV(j) is complete too.
@@ -31,13 +31,14 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "fastmath.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
 
 namespace h3 {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr int kTileRows = 128;  // query rows per CTA
 constexpr int kTileKeys = 128;  // keys per KV tile
 constexpr uint32_t kTmemCols = 256;
@@ -46,11 +47,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
+__device__ __forceinline__ float ex2(float x) { return ex2_mufu(x); }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -68,10 +65,11 @@ struct Layout {
   static constexpr int kK = kQ + kTileBytes;
   static constexpr int kV = kK + kTileBytes;
   static constexpr int kBars = kV + kTileBytes;
-  // barriers: q_full, k_full, k_empty, v_full, v_empty, s_full, p_full[2], o_half0, o_final, drain
-  static constexpr int kNumBars = 11;
+  // barriers: q_full, k_full, k_empty, v_full, v_empty, s_full, p_full[2], o_half0, o_final, drain, xchg[4]
+  static constexpr int kNumBars = 15;
   static constexpr int kMisc = kBars + kNumBars * 8;  // tmem base, abort flag, n_entries
-  static constexpr int kBitmaps = kMisc + 16;
+  static constexpr int kRed = kMisc + 16;             // partial row maxima / sums: float [2][2][128]
+  static constexpr int kBitmaps = kRed + 2 * 2 * 128 * 4;
   static int host_bytes(int n_blocks) {
     const int nwords = (n_blocks + 31) / 32;
     return 1024 /*alignment slack*/ + kBitmaps + 2 * nwords * 4 + ((n_blocks * 2 + 15) & ~15);
@@ -79,14 +77,17 @@ struct Layout {
 };
 
 struct Bars {
-  uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *o_half0, *o_final, *drain;
+  uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *o_half0, *o_final, *drain, *xchg;
 };
 
 // p_full[h]: P of half h of the current tile is in TMEM (one completion per
 // tile each, so a waiter is never more than one phase behind).
+// xchg[q]: the two softmax warps of TMEM lane quarter q have written their
+// partial row values (64 arrivals per exchange; neither warp can run more than
+// one exchange ahead of the other).
 __device__ __forceinline__ Bars carve_bars(uint8_t* base) {
   uint64_t* b = reinterpret_cast<uint64_t*>(base);
-  return Bars{b, b + 1, b + 2, b + 3, b + 4, b + 5, b + 6, b + 8, b + 9, b + 10};
+  return Bars{b, b + 1, b + 2, b + 3, b + 4, b + 5, b + 6, b + 8, b + 9, b + 10, b + 11};
 }
 
 // Bounded wait with CTA-wide abort.  On give-up: raise the CTA abort flag and
@@ -176,11 +177,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     mbar_init(bars.v_full, 1);
     mbar_init(bars.v_empty, 1);
     mbar_init(bars.s_full, 1);
-    mbar_init(bars.p_full, 128);
-    mbar_init(bars.p_full + 1, 128);
+    mbar_init(bars.p_full, 8);
+    mbar_init(bars.p_full + 1, 8);
     mbar_init(bars.o_half0, 1);
     mbar_init(bars.o_final, 1);
     mbar_init(bars.drain, 1);
+    for (int q = 0; q < 4; ++q) mbar_init(bars.xchg + q, 64);
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -347,13 +349,24 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   } else {
     // ------------------------------------------------------------ softmax
+    // Two threads per query row: warp w handles TMEM lanes [32 (w % 4), +32)
+    // and, inside every 64-key half, the 32 keys [32 part, 32 part + 32) with
+    // part = (w - 2) / 4.  The two threads of a row exchange their partial
+    // maxima through shared memory (one named barrier per lane quarter), so
+    // both apply the same running max; each rescales and finally normalises
+    // its half of O's columns.
     // tcgen05.ld/st are warp-collective (.sync.aligned): every branch that
     // guards one is made warp-uniform with __all_sync / __any_sync.
+    constexpr int kOCols = D / 2;  // O columns per thread
     const int quarter = warp & 3;
+    const int part = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;  // row within the tile == TMEM lane
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
     const uint32_t t_s = tmem_base + lane_addr;
-    const uint32_t t_o = tmem_base + lane_addr + kTmemO;
+    const uint32_t t_o = tmem_base + lane_addr + kTmemO + (uint32_t)(part * kOCols);
+    uint64_t* xbar = bars.xchg + quarter;
+    uint32_t n_xchg = 0;  // exchanges done (phase parity of xbar)
+    float* red = reinterpret_cast<float*>(smem + L::kRed);  // [2 slots][2 parts][128 rows]
     const int my_bit = 14 + (r >> 6);  // list bit of this row's query block
     const int qrow = qtile * kTileRows + r;
     const bool row_valid = qrow < p.S;
@@ -361,9 +374,19 @@ __global__ void __launch_bounds__(kThreads, 2)
     const float tq = pen_row ? p.times[qrow] : 0.0f;
     const float scale = p.scale_log2;
     float m = -INFINITY;  // running max, log2 units (upper bound of the true max)
-    float l = 0.0f;
+    float l = 0.0f;       // partial row sum over this thread's keys
     bool ok = true;
     for (int j = 0; ok && j < n_tiles; ++j) {
+      // this tile's two key blocks and their descriptors, fetched before the
+      // wait so the loads overlap it
+      uint32_t ents[2];
+      uint2 kds[2];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int idx = 2 * j + hh;
+        ents[hh] = idx < n_entries ? (uint32_t)list[idx] : 0u;
+        kds[hh] = ((ents[hh] >> my_bit) & 1u) ? __ldg(p.kv_desc + (ents[hh] & 0x3FFFu)) : make_uint2(0u, 0u);
+      }
       const bool got = wait_bar(bars.s_full, (uint32_t)j & 1u, p, abort_flag);
       if (!__all_sync(kFull, got)) {
         ok = false;
@@ -377,10 +400,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         float cpen = 0.0f;
         const int idx = 2 * j + hh;
         if (idx < n_entries) {
-          const uint32_t ent = list[idx];
+          const uint32_t ent = ents[hh];
           kblock = (int)(ent & 0x3FFFu);
           if ((ent >> my_bit) & 1u) {
-            const uint2 kd = p.kv_desc[kblock];
+            const uint2 kd = kds[hh];
             nv = (int)(kd.x & 0xFFu);
             const int kind = (int)((kd.x >> 8) & 3u);
             mode = 1;
@@ -392,32 +415,114 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
           }
         }
-        float sv[64];
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        const int col0 = part * 32;  // first key of this thread inside the half
+        float sv[32];
+        {
           uint32_t tmp[32];
           __syncwarp();
-          tmem_ld32(t_s + hh * 64 + c * 32, tmp);
+          tmem_ld32(t_s + hh * 64 + col0, tmp);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(tmp[i]);
+          for (int i = 0; i < 32; ++i) sv[i] = __uint_as_float(tmp[i]);
         }
-        float mx = -INFINITY;
+        float pmax = -INFINITY;
         if (mode != 0) {
           if (nv == 64) {
+            float mp[4];
 #pragma unroll
-            for (int i = 0; i < 64; ++i) mx = fmaxf(mx, sv[i]);
+            for (int a = 0; a < 4; ++a) mp[a] = fmaxf(sv[a], sv[a + 4]);
+#pragma unroll
+            for (int i = 8; i < 32; i += 8)
+#pragma unroll
+              for (int a = 0; a < 4; ++a) mp[a] = max3f(mp[a], sv[i + a], sv[i + 4 + a]);
+            pmax = fmaxf(max3f(mp[0], mp[1], mp[2]), mp[3]);
           } else {
 #pragma unroll
-            for (int i = 0; i < 64; ++i)
-              if (i < nv) mx = fmaxf(mx, sv[i]);
+            for (int i = 0; i < 32; ++i)
+              if (col0 + i < nv) pmax = fmaxf(pmax, sv[i]);
           }
         }
-        mx *= scale;
+        // combine the two partial maxima of the row (slot hh: a slot is
+        // rewritten only after the next exchange's barrier, which both threads
+        // pass after reading it)
+        red[(hh * 2 + part) * 128 + r] = pmax;
+        mbar_arrive(xbar);
+        const bool gotx = wait_bar(xbar, n_xchg & 1u, p, abort_flag);
+        ++n_xchg;
+        if (!__all_sync(kFull, gotx)) {
+          ok = false;
+          break;
+        }
+        const float mx = fmaxf(pmax, red[(hh * 2 + (part ^ 1)) * 128 + r]) * scale;
         // Conditional rescale: the running max only moves when it grows by
         // more than 2^8; below that the stale max keeps every probability <= 256.
         const bool grow = mx > m + kRescaleThreshold;
-        const bool o_rescale = grow && l > 0.0f;
+        const bool o_rescale = grow && m > -INFINITY;
+        const float m_old = m;
+        if (grow) m = mx;
+        // probabilities of this thread's 32 keys -> bf16 pairs into P columns
+        // [32 hh + 16 part, +16) (P(j) overwrites the first 64 columns of S)
+        float lt = 0.0f;
+        uint32_t packed[16];
+        if (mode == 0) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) packed[i] = 0u;
+        } else if (mode == 3) {
+          const int key0 = kblock * 64 + col0;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float pp[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int col = col0 + 2 * i + e;
+              float pen_k = 0.0f;
+              if (col < nv && p.seg[key0 + 2 * i + e] == kSegGuide)
+                pen_k = block_penalty_log2(tq, p.times[key0 + 2 * i + e], p);
+              pp[e] = col < nv ? ex2(fmaf(sv[2 * i + e], scale, -(m + pen_k))) : 0.0f;
+            }
+            lt += pp[0] + pp[1];
+            packed[i] = pack_bf16(pp[0], pp[1]);
+          }
+        } else if (nv == 64) {
+          // pairs in packed fp32: scale and offset by one f32x2 FMA; one pair
+          // in four takes 2^x on the FMA pipe, the rest on MUFU
+          const float off = -(m + cpen);
+          const uint64_t scale2 = f2_pack(scale, scale), off2 = f2_pack(off, off);
+          uint64_t acc2[2] = {f2_pack(0.0f, 0.0f), f2_pack(0.0f, 0.0f)};
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const uint64_t x2 = f2_fma(f2_pack(sv[2 * i], sv[2 * i + 1]), scale2, off2);
+            uint64_t p2;
+            if ((i & 3) == 3) {
+              p2 = ex2_poly2(x2);
+            } else {
+              float a, b;
+              f2_unpack(x2, a, b);
+              p2 = f2_pack(ex2(a), ex2(b));
+            }
+            acc2[i & 1] = f2_add(acc2[i & 1], p2);
+            float p0, p1;
+            f2_unpack(p2, p0, p1);
+            packed[i] = pack_bf16(p0, p1);
+          }
+          float a0, a1, b0, b1;
+          f2_unpack(acc2[0], a0, a1);
+          f2_unpack(acc2[1], b0, b1);
+          lt = (a0 + a1) + (b0 + b1);
+        } else {
+          const float off = -(m + cpen);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int col = col0 + 2 * i;
+            const float p0 = col < nv ? ex2(fmaf(sv[2 * i], scale, off)) : 0.0f;
+            const float p1 = col + 1 < nv ? ex2(fmaf(sv[2 * i + 1], scale, off)) : 0.0f;
+            lt += p0 + p1;
+            packed[i] = pack_bf16(p0, p1);
+          }
+        }
+        __syncwarp();
+        tmem_st16(t_s + hh * 32 + part * 16, packed);
+        // O rescale (rare), after the scores are dead to keep registers low
         float alpha = 1.0f;
         if (__any_sync(kFull, o_rescale)) {
           // Half 0: O is stable (PV(j-1) completed before S(j) did).  Half 1:
@@ -430,9 +535,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             tc_fence_after();
           }
-          alpha = o_rescale ? ex2(m - mx) : 1.0f;
+          alpha = o_rescale ? ex2(m_old - m) : 1.0f;
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < kOCols / 32; ++c) {
             uint32_t tmp[32];
             __syncwarp();
             tmem_ld32(t_o + c * 32, tmp);
@@ -442,69 +547,30 @@ __global__ void __launch_bounds__(kThreads, 2)
             tmem_st32(t_o + c * 32, tmp);
           }
         }
-        if (grow) m = mx;
-        // probabilities -> bf16 pairs into columns [32 hh, 32 hh + 32) of S
-        float lt = 0.0f;
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t packed[16];
-          if (mode == 0) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) packed[i] = 0u;
-          } else if (mode == 3) {
-            const int key0 = kblock * 64 + c * 32;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              float pp[2];
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                const int col = c * 32 + 2 * i + e;
-                float pen_k = 0.0f;
-                if (col < nv && p.seg[key0 + 2 * i + e] == kSegGuide)
-                  pen_k = block_penalty_log2(tq, p.times[key0 + 2 * i + e], p);
-                pp[e] = col < nv ? ex2(fmaf(sv[col], scale, -(m + pen_k))) : 0.0f;
-              }
-              lt += pp[0] + pp[1];
-              packed[i] = pack_bf16(pp[0], pp[1]);
-            }
-          } else if (nv == 64) {
-            const float off = -(m + cpen);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float p0 = ex2(fmaf(sv[c * 32 + 2 * i], scale, off));
-              const float p1 = ex2(fmaf(sv[c * 32 + 2 * i + 1], scale, off));
-              lt += p0 + p1;
-              packed[i] = pack_bf16(p0, p1);
-            }
-          } else {
-            const float off = -(m + cpen);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int col = c * 32 + 2 * i;
-              const float p0 = col < nv ? ex2(fmaf(sv[col], scale, off)) : 0.0f;
-              const float p1 = col + 1 < nv ? ex2(fmaf(sv[col + 1], scale, off)) : 0.0f;
-              lt += p0 + p1;
-              packed[i] = pack_bf16(p0, p1);
-            }
-          }
-          __syncwarp();
-          tmem_st16(t_s + hh * 32 + c * 16, packed);
-        }
         l = l * alpha + lt;
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bars.p_full + hh);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars.p_full + hh);  // one arrival per softmax warp
       }
     }
     // ---------------------------------------------------------- epilogue
     bool fin = __all_sync(kFull, ok) && n_tiles > 0;
-    if (fin) fin = wait_bar(bars.o_final, 0, p, abort_flag);
+    // total row sum: slot 0 is free here (its last reader passed the barrier
+    // of the final half-1 exchange before this thread did)
+    if (fin) {
+      red[part * 128 + r] = l;
+      mbar_arrive(xbar);
+      fin = wait_bar(xbar, n_xchg & 1u, p, abort_flag);
+      if (fin) l += red[(part ^ 1) * 128 + r];
+      if (fin) fin = wait_bar(bars.o_final, 0, p, abort_flag);
+    }
     if (__all_sync(kFull, fin)) {
       tc_fence_after();
       const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
-      uint16_t* orow = p.o + ((size_t)head * p.S + (row_valid ? qrow : 0)) * D;
+      uint16_t* orow = p.o + ((size_t)head * p.S + (row_valid ? qrow : 0)) * D + part * kOCols;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < kOCols / 32; ++c) {
         uint32_t tmp[32];
         __syncwarp();
         tmem_ld32(t_o + c * 32, tmp);
@@ -520,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             dst[v] = make_uint4(outw[4 * v], outw[4 * v + 1], outw[4 * v + 2], outw[4 * v + 3]);
         }
       }
-      if (row_valid && p.lse != nullptr) p.lse[(size_t)head * p.S + qrow] = (m + __log2f(l)) * kLn2;
+      if (row_valid && part == 0 && p.lse != nullptr) p.lse[(size_t)head * p.S + qrow] = (m + __log2f(l)) * kLn2;
     }
   }
 

@@ -49,5 +49,6 @@ cudaError_t launch_route(const float* qp, const float* kp, int32_t* kv_sel, int 
                          int k, int first_video_block, cudaStream_t stream);
 
 cudaError_t launch_selftest_timeout(int* status, uint32_t polls, cudaStream_t stream);
+cudaError_t launch_selftest_exp2(const float* x, float* y, int n_pairs, cudaStream_t stream);
 
 }  // namespace h3

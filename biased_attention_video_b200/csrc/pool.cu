@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
+#include "fastmath.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -108,7 +109,21 @@ __global__ void selftest_timeout_kernel(int* status, uint32_t polls) {
   }
 }
 
+__global__ void selftest_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, int n_pairs) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n_pairs) return;
+  float a, b;
+  f2_unpack(ex2_poly2(f2_pack(x[2 * i], x[2 * i + 1])), a, b);
+  y[2 * i] = a;
+  y[2 * i + 1] = b;
+}
+
 }  // namespace
+
+cudaError_t launch_selftest_exp2(const float* x, float* y, int n_pairs, cudaStream_t stream) {
+  if (n_pairs > 0) selftest_exp2_kernel<<<(n_pairs + 255) / 256, 256, 0, stream>>>(x, y, n_pairs);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_pool(const uint16_t* x0, float* out0, const uint16_t* x1, float* out1, int H, int S, int d,
                         int first_block, int n_out, cudaStream_t stream) {

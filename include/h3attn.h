@@ -186,6 +186,12 @@ H3ATTN_API int h3attn_check(void* ws, void* stream);
  * H3ATTN_ETIMEOUT in the status word when it gives up.  No other work. */
 H3ATTN_API int h3attn_selftest_timeout(void* ws, uint32_t polls, void* stream);
 
+/* Self-test of the softmax's FMA-pipe exponential: y[i] = 2^x[i] computed
+ * the way the attention kernel computes one pair in four of its
+ * probabilities (inputs below -125 are clamped to -125).  x, y: float32 [n]
+ * device, n even, 8-byte aligned. */
+H3ATTN_API int h3attn_selftest_exp2(const float* x, float* y, int n, void* stream);
+
 /* Static description of a status code (never NULL). */
 H3ATTN_API const char* h3attn_strerror(int status);
 
