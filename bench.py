@@ -354,7 +354,7 @@ def run_ours(args, rank, world, local_rank):
                      "peak_source": f"{peak_kind} bf16_tflops_sustained"},
         "routing": {"ms": route_ms, "bytes_read": route_bytes, "gbs": route_bytes / (route_ms * 1e-3) / 1e9,
                     "hbm_peak_gbs": peaks["hbm_gbs"]},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 5 * args.steps,  # pool_split, score_gemm, topk, kv_desc, attn
         "clocks": clk,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms / args.steps},

@@ -10,9 +10,6 @@
 #include "h3attn.h"
 #include "kernels.cuh"
 
-namespace h3 {
-size_t route_smem_bytes(int d, int n_video);
-}
 
 namespace {
 
@@ -27,15 +24,15 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 struct WsLayout {
-  size_t desc, qp, kp, total;
+  size_t desc, route, total;
 };
 
+// status word | per-key-block descriptors | routing scratch
 WsLayout ws_layout(int H, int d, int n_blocks, int n_video) {
   WsLayout w;
   w.desc = kStatusBytes;
-  w.qp = w.desc + align_up((size_t)n_blocks * sizeof(uint2));
-  w.kp = w.qp + align_up((size_t)H * n_video * d * sizeof(float));
-  w.total = w.kp + align_up((size_t)H * n_video * d * sizeof(float));
+  w.route = w.desc + align_up((size_t)n_blocks * sizeof(uint2));
+  w.total = w.route + (n_video > 0 ? h3::route_scratch_layout(H, d, n_video).total : 0);
   return w;
 }
 
@@ -63,18 +60,9 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 [H][S][d] viewed as 3-D {d, S, H}; box {64, 64, 1}, 128-byte swizzle,
-// rows past S (and past the head) read as zero.
+// bf16 [H][S][d] viewed as 3-D {d, S, H}; box {64, 64, 1}
 bool make_map(CUtensorMap* m, const void* base, int H, int S, int d) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)S, (cuuint64_t)H};
-  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)S * d * 2};
-  cuuint32_t box[3] = {64, 64, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return h3::encode_bf16_3d(m, base, (uint64_t)d, (uint64_t)S, (uint64_t)H, 64, 64);
 }
 
 bool finite_nonneg(float x) { return std::isfinite(x) && x >= 0.0f; }
@@ -141,6 +129,21 @@ int forward_impl(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, 
 
 }  // namespace
 
+namespace h3 {
+bool encode_bf16_3d(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2, uint32_t box0,
+                    uint32_t box1) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {dim0, dim1, dim2};
+  cuuint64_t strides[2] = {dim0 * 2, dim0 * dim1 * 2};
+  cuuint32_t box[3] = {box0, box1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+}  // namespace h3
+
 extern "C" {
 
 int h3attn_plan_init(h3attn_plan* plan, int H, int S, int d, int block, float sparsity, const uint8_t* seg_host) {
@@ -205,14 +208,9 @@ int h3attn_route(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, 
     return H3ATTN_EALIGN;
   if (h3::route_smem_bytes(plan->d, plan->n_video_blocks) > (size_t)kMaxSmem) return H3ATTN_EUNSUPPORTED;
   uint8_t* wsb = static_cast<uint8_t*>(ws);
-  float* qp = reinterpret_cast<float*>(wsb + w.qp);
-  float* kp = reinterpret_cast<float*>(wsb + w.kp);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (h3::launch_pool(q, qp, k, kp, plan->H, plan->S, plan->d, plan->first_video_block, plan->n_video_blocks, st) !=
-      cudaSuccess)
-    return H3ATTN_ECUDA;
-  if (h3::launch_route(qp, kp, kv_sel, plan->H, plan->d, plan->n_video_blocks, plan->k, plan->first_video_block,
-                       st) != cudaSuccess)
+  if (h3::launch_route_pipeline(q, k, kv_sel, plan->H, plan->S, plan->d, plan->first_video_block,
+                                plan->n_video_blocks, plan->k, wsb + w.route, reinterpret_cast<int*>(wsb),
+                                static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return H3ATTN_ECUDA;
   return H3ATTN_OK;
 }

@@ -44,9 +44,23 @@ cudaError_t launch_kv_desc(const uint8_t* seg, const float* times, int S, int n_
 cudaError_t launch_pool(const uint16_t* x0, float* out0, const uint16_t* x1, float* out1, int H, int S,
                         int d, int first_block, int n_out, cudaStream_t stream);
 
-// pooled scores of video query blocks vs video key blocks + top-k, per head
-cudaError_t launch_route(const float* qp, const float* kp, int32_t* kv_sel, int H, int d, int n_video,
-                         int k, int first_video_block, cudaStream_t stream);
+// bf16 tensor [dim2][dim1][dim0] (dim0 contiguous) as a 3-D TMA map with a
+// {box0, box1, 1} box and 128-byte swizzle; out-of-range elements read as zero
+bool encode_bf16_3d(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2, uint32_t box0,
+                    uint32_t box1);
+
+// Routing scratch (byte offsets): two-part bf16 pooled centroids of Q and K
+// [H][n_video][3 d] and the fp32 score matrix [H][n_video][ldc].
+struct RouteScratch {
+  size_t qs, ks, scores, ldc, total;
+};
+RouteScratch route_scratch_layout(int H, int d, int n_video);
+size_t route_smem_bytes(int d, int n_video);  // shared memory of one top-k warp
+
+// pool + split, tensor-core pooled scores, top-k: kv_sel[H][n_video][k]
+cudaError_t launch_route_pipeline(const uint16_t* q, const uint16_t* k, int32_t* kv_sel, int H, int S, int d,
+                                  int first_video_block, int n_video, int kk, void* scratch, int* status,
+                                  cudaStream_t stream);
 
 cudaError_t launch_selftest_timeout(int* status, uint32_t polls, cudaStream_t stream);
 cudaError_t launch_selftest_exp2(const float* x, float* y, int n_pairs, cudaStream_t stream);

@@ -2,186 +2,415 @@
 // is scored against every key block with one small pooled matmul and only the
 // top 1 - sparsity_ratio fraction is kept).
 //
-// One CTA scores kQB video query blocks of one head against all video key
-// blocks (fp32 dot products of the pooled centroids, kept in shared memory),
-// then each warp selects the k best of a row by a 4-pass radix select on the
-// order-preserving integer image of the fp32 score, ties to the lower block,
-// and writes the chosen blocks in ascending order.  The 1/sqrt(d) scale is a
-// positive constant and does not change the order, so it is not applied.
+// Three kernels:
+//  1. pool_split_kernel: mean of every video block of Q and K (fp32 sums of the
+//     bf16 rows), written as two bf16 parts x = hi + lo (hi = bf16(x),
+//     lo = bf16(x - hi)), rows [hi | hi | lo] for Q and [hi | lo | hi] for K.
+//  2. score_gemm_kernel: per head, scores = Qs . Ks^T over the concatenated
+//     3d-long rows, i.e. Qh.Kh + Qh.Kl + Ql.Kh -- the fp32 products of the
+//     pooled centroids up to the dropped Ql.Kl term and the residual of the
+//     two-part split (relative 2^-16 per product), on the tensor cores
+//     (tcgen05.mma kind::f16, fp32 accumulation in TMEM).
+//  3. topk_kernel: one warp per (head, query block): the k best key blocks,
+//     ties to the lower block, listed in ascending order.
+// The 1/sqrt(d) logit scale is a positive constant and does not change the
+// order, so it is not applied.
+#include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cstdint>
 
 #include "kernels.cuh"
+#include "ptx.cuh"
 
 namespace h3 {
 namespace {
 
-constexpr int kQB = 16;      // query blocks per CTA
-constexpr int kKC = 64;      // key blocks per shared-memory chunk
-constexpr int kThreads = 256;
-
-__device__ __forceinline__ uint32_t order_key(float f) {
-  const uint32_t u = __float_as_uint(f);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+__device__ __forceinline__ void add_bf16x8(float (&acc)[8], uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc[2 * i] += __uint_as_float(w[i] << 16);
+    acc[2 * i + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
+  }
 }
 
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// One warp per (tensor, head, video block).  Output row layout (3d bf16):
+// Q: [hi | hi | lo], K: [hi | lo | hi] so that the row dot product of the two
+// concatenations is Qh.Kh + Qh.Kl + Ql.Kh.
 template <int D>
-__global__ void __launch_bounds__(kThreads) route_kernel(const float* __restrict__ qp, const float* __restrict__ kp,
-                                                         int32_t* __restrict__ sel, int n_video, int k,
-                                                         int first_video_block) {
-  constexpr int kPad = D + 4;  // float4-aligned row pitch, conflict-free 16-byte reads
-  extern __shared__ float4 smem4[];
-  float* qs = reinterpret_cast<float*>(smem4);           // [kQB][kPad]
-  float* ks = qs + kQB * kPad;                           // [kKC][kPad]
-  float* scores = ks + kKC * kPad;                       // [kQB][n_video]
-  uint32_t* hist = reinterpret_cast<uint32_t*>(scores + kQB * n_video);  // [8 warps][256]
-
-  const int h = blockIdx.y;
-  const int i0 = blockIdx.x * kQB;
-  const int nq = min(kQB, n_video - i0);
-  const int tid = threadIdx.x;
-  const float* qph = qp + (size_t)h * n_video * D;
-  const float* kph = kp + (size_t)h * n_video * D;
-
-  for (int idx = tid; idx < kQB * (D / 4); idx += kThreads) {
-    const int r = idx / (D / 4), c4 = idx % (D / 4);
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (r < nq) v = reinterpret_cast<const float4*>(qph + (size_t)(i0 + r) * D)[c4];
-    reinterpret_cast<float4*>(qs + r * kPad)[c4] = v;
-  }
-
-  // ---- scores: thread (ty, tx) computes query block ty x key blocks tx + 16 e, e < 4
-  const int ty = tid >> 4, tx = tid & 15;
-  for (int j0 = 0; j0 < n_video; j0 += kKC) {
-    __syncthreads();
-    const int nk = min(kKC, n_video - j0);
-    for (int idx = tid; idx < kKC * (D / 4); idx += kThreads) {
-      const int r = idx / (D / 4), c4 = idx % (D / 4);
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r < nk) v = reinterpret_cast<const float4*>(kph + (size_t)(j0 + r) * D)[c4];
-      reinterpret_cast<float4*>(ks + r * kPad)[c4] = v;
-    }
-    __syncthreads();
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const float4* qrow = reinterpret_cast<const float4*>(qs + ty * kPad);
-#pragma unroll 4
-    for (int c4 = 0; c4 < D / 4; ++c4) {
-      const float4 a = qrow[c4];
+__global__ void __launch_bounds__(256) pool_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
+                                                         uint16_t* __restrict__ qs, uint16_t* __restrict__ ks, int H,
+                                                         int S, int first_block, int n_video) {
+  constexpr int kLanesPerRow = D / 8;
+  constexpr int kRowsPerPass = 32 / kLanesPerRow;
+  constexpr int kPasses = kBlock / kRowsPerPass;
+  const long long warp_id = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const long long per_tensor = (long long)H * n_video;
+  if (warp_id >= 2 * per_tensor) return;
+  const int t = (int)(warp_id / per_tensor);
+  const long long rem = warp_id % per_tensor;
+  const int h = (int)(rem / n_video);
+  const int vb = (int)(rem % n_video);
+  const int row0 = (first_block + vb) * kBlock;
+  const int nrows = min(kBlock, S - row0);
+  const int chunk = lane % kLanesPerRow;
+  const int rsub = lane / kLanesPerRow;
+  const uint16_t* x = t == 0 ? q : k;
+  const uint4* src = reinterpret_cast<const uint4*>(x + ((size_t)h * S + row0) * D) + chunk;
+  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  if (nrows == kBlock) {
+    constexpr int kBatch = 8;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float4 b = reinterpret_cast<const float4*>(ks + (tx + 16 * e) * kPad)[c4];
-        acc[e] = fmaf(a.x, b.x, acc[e]);
-        acc[e] = fmaf(a.y, b.y, acc[e]);
-        acc[e] = fmaf(a.z, b.z, acc[e]);
-        acc[e] = fmaf(a.w, b.w, acc[e]);
+    for (int i0 = 0; i0 < kPasses; i0 += kBatch) {
+      uint4 v[kBatch];
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i)
+        v[i] = __ldg(src + (size_t)((i0 + i) * kRowsPerPass + rsub) * kLanesPerRow);
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) add_bf16x8(acc, v[i]);
+    }
+  } else {
+    for (int r = rsub; r < nrows; r += kRowsPerPass) add_bf16x8(acc, __ldg(src + (size_t)r * kLanesPerRow));
+  }
+#pragma unroll
+  for (int o = kLanesPerRow; o < 32; o <<= 1)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xFFFFFFFFu, acc[i], o);
+  if (rsub == 0) {
+    const float inv = 1.0f / (float)nrows;
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float a = acc[2 * i] * inv, b = acc[2 * i + 1] * inv;
+      const float ah = __bfloat162float(__float2bfloat16_rn(a)), bh = __bfloat162float(__float2bfloat16_rn(b));
+      hw[i] = bf16x2_bits(ah, bh);
+      lw[i] = bf16x2_bits(a - ah, b - bh);
+    }
+    const uint4 hv = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    const uint4 lv = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    uint16_t* dst_row = (t == 0 ? qs : ks) + ((size_t)h * n_video + vb) * (3 * D) + chunk * 8;
+    uint4* d0 = reinterpret_cast<uint4*>(dst_row);
+    uint4* d1 = reinterpret_cast<uint4*>(dst_row + D);
+    uint4* d2 = reinterpret_cast<uint4*>(dst_row + 2 * D);
+    *d0 = hv;
+    *d1 = t == 0 ? hv : lv;
+    *d2 = t == 0 ? lv : hv;
+  }
+}
+
+
+// ----------------------------------------------------------- score GEMM
+constexpr int kGemmThreads = 128;
+constexpr int kGM = 128;                    // query blocks per tile (UMMA M)
+constexpr int kGN = 256;                    // key blocks per tile (UMMA N)
+constexpr int kGStages = 2;
+constexpr int kGStageA = kGM * 128;         // one 64-element (128-byte) K chunk of A
+constexpr int kGStageB = kGN * 128;
+constexpr int kGStageBytes = kGStageA + kGStageB;
+constexpr int kGBars = kGStages * kGStageBytes;
+constexpr int kGSmem = 1024 + kGBars + 64;
+
+__device__ __forceinline__ bool gemm_wait(uint64_t* bar, uint32_t parity, int* status) {
+  uint64_t t0 = 0;
+  for (uint32_t i = 0;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 1023u) == 1023u) {
+      uint64_t now;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
+      if (t0 == 0) t0 = now;
+      if (now - t0 > 2000000000ull) {
+        if (status != nullptr) atomicCAS(status, 0, kStatusTimeout);
+        return false;
       }
     }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int j = tx + 16 * e;
-      if (ty < nq && j < nk) scores[ty * n_video + j0 + j] = acc[e];
-    }
   }
+}
+
+// scores[h][i][j] (row pitch ldc floats) for query blocks i in [m0, m0 + 128)
+// and key blocks j in [n0, n0 + 256) of head h.  Rows past n_video read as
+// zero (TMA fill) and are not stored.
+__global__ void __launch_bounds__(kGemmThreads, 2)
+    score_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                      float* __restrict__ scores, int n_video, int ldc, int n_chunks, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGBars);
+  uint64_t* empty = full + kGStages;
+  uint64_t* done = empty + kGStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n0 = blockIdx.x * kGN, m0 = blockIdx.y * kGM, h = blockIdx.z;
+  if (tid == 0) {
+    for (int s = 0; s < kGStages; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    mbar_init(done, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
 
-  // ---- top-k per row: radix select of the k-th largest key, then an ordered sweep
-  const int warp = tid >> 5, lane = tid & 31;
-  uint32_t* wh = hist + warp * 256;
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  for (int row = warp; row < nq; row += kThreads / 32) {
-    const float* s = scores + row * n_video;
-    uint32_t prefix = 0, pmask = 0;
-    int need = k;
+  if (warp == 0 && lane == 0) {
+    uint32_t issued[kGStages] = {0, 0};
+    for (int c = 0; c < n_chunks; ++c) {
+      const int s = c % kGStages;
+      const uint32_t ph = (uint32_t)(c / kGStages) & 1u;
+      if (!gemm_wait(empty + s, ph ^ 1u, status)) break;
+      uint8_t* st = smem + s * kGStageBytes;
+      mbar_arrive_expect_tx(full + s, kGStageBytes);
+      tma_load_3d(st, &tm_a, full + s, c * 64, m0, h);
+      tma_load_3d(st + kGStageA, &tm_b, full + s, c * 64, n0, h);
+      ++issued[s];
+    }
+    for (int s = 0; s < kGStages; ++s)
+      if (issued[s]) gemm_wait(full + s, (issued[s] - 1) & 1u, status);
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t kIdesc = idesc_bf16_f32(kGM, kGN, 0, 0);
+    for (int c = 0; c < n_chunks; ++c) {
+      const int s = c % kGStages;
+      const uint32_t ph = (uint32_t)(c / kGStages) & 1u;
+      if (!gemm_wait(full + s, ph, status)) break;
+      tc_fence_after();
+      const uint32_t a = smem_u32(smem + s * kGStageBytes), b = a + kGStageA;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        umma_ss(tmem, sw128_desc(a + kk * 32, 16, 1024), sw128_desc(b + kk * 32, 16, 1024), kIdesc,
+                (c > 0 || kk > 0) ? 1u : 0u);
+      umma_commit(empty + s);
+    }
+    umma_commit(done);
+  }
+  // epilogue: thread = query block row; TMEM -> fp32 scores
+  const bool got = gemm_wait(done, 0, status);
+  if (__all_sync(0xFFFFFFFFu, got)) {
+    tc_fence_after();
+    const int i = m0 + warp * 32 + lane;
+    float* row = scores + ((size_t)h * n_video + (i < n_video ? i : 0)) * ldc;
 #pragma unroll 1
-    for (int shift = 24; shift >= 0; shift -= 8) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) wh[lane * 8 + i] = 0;
+    for (int cc = 0; cc < kGN / 32; ++cc) {
+      uint32_t v[32];
       __syncwarp();
-      for (int j = lane; j < n_video; j += 32) {
-        const uint32_t key = order_key(s[j]);
-        if ((key & pmask) == prefix) atomicAdd(wh + ((key >> shift) & 255u), 1u);
-      }
-      __syncwarp();
-      // lane l holds digits 255-8l .. 248-8l (descending)
-      uint32_t c[8];
-      uint32_t sum = 0;
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + cc * 32, v);
+      tmem_wait_ld();
+      const int j0 = n0 + cc * 32;
+      if (i < n_video && j0 < n_video) {
+        if (j0 + 32 <= n_video) {
+          float4* dst = reinterpret_cast<float4*>(row + j0);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        c[e] = wh[255 - 8 * lane - e];
-        sum += c[e];
-      }
-      uint32_t incl = sum;
+          for (int t = 0; t < 8; ++t)
+            dst[t] = make_float4(__uint_as_float(v[4 * t]), __uint_as_float(v[4 * t + 1]), __uint_as_float(v[4 * t + 2]),
+                                 __uint_as_float(v[4 * t + 3]));
+        } else {
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      const uint32_t excl = incl - sum;
-      const bool here = excl < (uint32_t)need && (uint32_t)need <= incl;
-      const uint32_t who = __ballot_sync(0xFFFFFFFFu, here);
-      const int src = __ffs(who) - 1;
-      uint32_t digit = 0, greater = 0;
-      if (here) {
-        uint32_t cum = excl;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          if (cum + c[e] >= (uint32_t)need) {
-            digit = 255u - 8u * lane - e;
-            greater = cum;
-            break;
-          }
-          cum += c[e];
+          for (int t = 0; t < 32; ++t)
+            if (j0 + t < n_video) row[j0 + t] = __uint_as_float(v[t]);
         }
       }
-      digit = __shfl_sync(0xFFFFFFFFu, digit, src);
-      greater = __shfl_sync(0xFFFFFFFFu, greater, src);
-      need -= (int)greater;
-      prefix |= digit << shift;
-      pmask |= 255u << shift;
-      __syncwarp();
     }
-    // keys > prefix are taken; `need` keys == prefix, the lowest blocks first
-    int32_t* dst = sel + ((size_t)blockIdx.y * n_video + i0 + row) * k;
-    int pos = 0, eq_seen = 0;
-    for (int jb = 0; jb < n_video; jb += 32) {
-      const int j = jb + lane;
-      const uint32_t key = j < n_video ? order_key(s[j]) : 0u;
-      const bool gt = j < n_video && key > prefix;
-      const bool eq = j < n_video && key == prefix;
-      const uint32_t eqm = __ballot_sync(0xFFFFFFFFu, eq);
-      const bool take = gt || (eq && eq_seen + __popc(eqm & lt_mask) < need);
-      const uint32_t tm = __ballot_sync(0xFFFFFFFFu, take);
-      const int slot = pos + __popc(tm & lt_mask);
-      if (take && slot < k) dst[slot] = first_video_block + j;
-      pos += __popc(tm);
-      eq_seen += __popc(eqm);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+
+// ----------------------------------------------------------------- top-k
+// Per-warp shared memory (32-bit words): the row's scores (ldc), a 256-bin
+// histogram, candidate indices (16-bit) and a bitmap of chosen candidates.
+__host__ __device__ __forceinline__ int topk_warp_words(int n_video, int ldc) {
+  return (ldc + 256 + (n_video + 1) / 2 + (n_video + 31) / 32 + 3) & ~3;
+}
+
+// One warp per (head, video query block).  Selection: the row is binned
+// linearly between its minimum and maximum (a monotone map, equal scores share
+// a bin); the bin holding the k-th best score is found from the top of a
+// 256-bin histogram; every score in a higher bin is taken, and the candidates
+// in that bin are ranked exactly by (score descending, block ascending).
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ scores, int32_t* __restrict__ sel,
+                                                   int rows, int n_video, int ldc, int k, int first_video_block) {
+  extern __shared__ float4 tk_smem4[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (row >= rows) return;  // warp-uniform
+  const int words = topk_warp_words(n_video, ldc);
+  uint32_t* base = reinterpret_cast<uint32_t*>(tk_smem4) + (size_t)warp * words;
+  float* s = reinterpret_cast<float*>(base);
+  uint32_t* hist = base + ldc;
+  uint16_t* cand = reinterpret_cast<uint16_t*>(hist + 256);
+  uint32_t* chosen = hist + 256 + (n_video + 1) / 2;
+  const unsigned full = 0xFFFFFFFFu;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+
+  const float* src = scores + (size_t)row * ldc;
+  for (int j = lane * 4; j < n_video; j += 128) {
+    const float4 v = *reinterpret_cast<const float4*>(src + j);
+    *reinterpret_cast<float4*>(s + j) = v;
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) hist[lane * 8 + i] = 0u;
+  for (int w = lane; w < (n_video + 31) / 32; w += 32) chosen[w] = 0u;
+  __syncwarp();
+  float lo = INFINITY, hi = -INFINITY;
+  for (int j = lane; j < n_video; j += 32) {
+    lo = fminf(lo, s[j]);
+    hi = fmaxf(hi, s[j]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(full, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(full, hi, o));
+  }
+  const float bscale = hi > lo ? 256.0f / (hi - lo) : 0.0f;
+  auto bin_of = [&](float x) -> int { return min(255, (int)((x - lo) * bscale)); };
+  for (int j = lane; j < n_video; j += 32) atomicAdd(hist + bin_of(s[j]), 1u);
+  __syncwarp();
+  // bin T holding the k-th best: lane l owns bins 255-8l .. 248-8l (descending)
+  uint32_t c[8], sum = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    c[e] = hist[255 - 8 * lane - e];
+    sum += c[e];
+  }
+  uint32_t incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(full, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const uint32_t excl = incl - sum;
+  const bool here = excl < (uint32_t)k && (uint32_t)k <= incl;
+  const int src_lane = __ffs(__ballot_sync(full, here)) - 1;
+  int tbin = 0;
+  uint32_t greater = 0;
+  if (here) {
+    uint32_t cum = excl;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      if (cum + c[e] >= (uint32_t)k) {
+        tbin = 255 - 8 * lane - e;
+        greater = cum;
+        break;
+      }
+      cum += c[e];
     }
+  }
+  tbin = __shfl_sync(full, tbin, src_lane);
+  greater = __shfl_sync(full, greater, src_lane);
+  const int need = k - (int)greater;
+  // candidates (scores in bin tbin), gathered in ascending block order
+  int n_cand = 0;
+  for (int jb = 0; jb < n_video; jb += 32) {
+    const int j = jb + lane;
+    const bool is_c = j < n_video && bin_of(s[j]) == tbin;
+    const uint32_t m = __ballot_sync(full, is_c);
+    if (is_c) cand[n_cand + __popc(m & lt_mask)] = (uint16_t)j;
+    n_cand += __popc(m);
+  }
+  __syncwarp();
+  // exact rank among candidates: (score descending, block ascending)
+  for (int e = lane; e < n_cand; e += 32) {
+    const int je = cand[e];
+    const float ve = s[je];
+    int rank = 0;
+    for (int f = 0; f < n_cand; ++f) {
+      const int jf = cand[f];
+      const float vf = s[jf];
+      rank += (vf > ve || (vf == ve && jf < je)) ? 1 : 0;
+    }
+    if (rank < need) atomicOr(chosen + (je >> 5), 1u << (je & 31));
+  }
+  __syncwarp();
+  int32_t* dst = sel + (size_t)row * k;
+  int pos = 0;
+  for (int jb = 0; jb < n_video; jb += 32) {
+    const int j = jb + lane;
+    bool take = false;
+    if (j < n_video) {
+      const int b = bin_of(s[j]);
+      take = b > tbin || (b == tbin && ((chosen[j >> 5] >> (j & 31)) & 1u));
+    }
+    const uint32_t m = __ballot_sync(full, take);
+    const int slot = pos + __popc(m & lt_mask);
+    if (take && slot < k) dst[slot] = first_video_block + j;
+    pos += __popc(m);
   }
 }
 
 }  // namespace
 
-cudaError_t launch_route(const float* qp, const float* kp, int32_t* kv_sel, int H, int d, int n_video, int k,
-                         int first_video_block, cudaStream_t stream) {
-  const int pad = d + 4;
-  const size_t smem = sizeof(float) * ((size_t)kQB * pad + (size_t)kKC * pad + (size_t)kQB * n_video) +
-                      sizeof(uint32_t) * 8 * 256;
-  dim3 grid((n_video + kQB - 1) / kQB, H);
-  if (d == 64) {
-    cudaError_t e = cudaFuncSetAttribute(route_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    route_kernel<64><<<grid, kThreads, smem, stream>>>(qp, kp, kv_sel, n_video, k, first_video_block);
-  } else {
-    cudaError_t e = cudaFuncSetAttribute(route_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    route_kernel<128><<<grid, kThreads, smem, stream>>>(qp, kp, kv_sel, n_video, k, first_video_block);
-  }
-  return cudaGetLastError();
+RouteScratch route_scratch_layout(int H, int d, int n_video) {
+  RouteScratch r;
+  const size_t split = (size_t)H * n_video * 3 * d * sizeof(uint16_t);
+  r.qs = 0;
+  r.ks = (split + 255) / 256 * 256;
+  r.scores = r.ks + (split + 255) / 256 * 256;
+  r.ldc = (n_video + 3) & ~3;
+  r.total = r.scores + ((size_t)H * n_video * r.ldc * sizeof(float) + 255) / 256 * 256;
+  return r;
 }
 
 size_t route_smem_bytes(int d, int n_video) {
-  return sizeof(float) * ((size_t)kQB * (d + 4) + (size_t)kKC * (d + 4) + (size_t)kQB * n_video) +
-         sizeof(uint32_t) * 8 * 256;
+  (void)d;
+  return sizeof(uint32_t) * (size_t)topk_warp_words(n_video, (n_video + 3) & ~3);
+}
+
+cudaError_t launch_route_pipeline(const uint16_t* q, const uint16_t* k, int32_t* kv_sel, int H, int S, int d,
+                                  int first_video_block, int n_video, int kk, void* scratch, int* status,
+                                  cudaStream_t stream) {
+  const RouteScratch r = route_scratch_layout(H, d, n_video);
+  uint8_t* base = static_cast<uint8_t*>(scratch);
+  uint16_t* qs = reinterpret_cast<uint16_t*>(base + r.qs);
+  uint16_t* ks = reinterpret_cast<uint16_t*>(base + r.ks);
+  float* sc = reinterpret_cast<float*>(base + r.scores);
+  // 1. pool + split
+  const long long warps = 2LL * H * n_video;
+  const unsigned pgrid = (unsigned)((warps + 7) / 8);
+  if (d == 64)
+    pool_split_kernel<64><<<pgrid, 256, 0, stream>>>(q, k, qs, ks, H, S, first_video_block, n_video);
+  else
+    pool_split_kernel<128><<<pgrid, 256, 0, stream>>>(q, k, qs, ks, H, S, first_video_block, n_video);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // 2. scores on the tensor cores
+  CUtensorMap ta, tb;
+  if (!encode_bf16_3d(&ta, qs, 3 * d, n_video, H, 64, kGM) || !encode_bf16_3d(&tb, ks, 3 * d, n_video, H, 64, kGN))
+    return cudaErrorInvalidValue;
+  e = cudaFuncSetAttribute(score_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmem);
+  if (e != cudaSuccess) return e;
+  dim3 ggrid((n_video + kGN - 1) / kGN, (n_video + kGM - 1) / kGM, H);
+  score_gemm_kernel<<<ggrid, kGemmThreads, kGSmem, stream>>>(ta, tb, sc, n_video, (int)r.ldc, 3 * d / 64, status);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // 3. top-k per (head, query block)
+  const int words = topk_warp_words(n_video, (int)r.ldc);
+  int wpc = (int)((200 * 1024) / (words * 4));
+  wpc = wpc < 1 ? 1 : (wpc > 8 ? 8 : wpc);
+  const size_t tsmem = (size_t)wpc * words * 4;
+  e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsmem);
+  if (e != cudaSuccess) return e;
+  const int rows = H * n_video;
+  topk_kernel<<<(rows + wpc - 1) / wpc, wpc * 32, tsmem, stream>>>(sc, kv_sel, rows, n_video, (int)r.ldc, kk,
+                                                                   first_video_block);
+  return cudaGetLastError();
 }
 
 }  // namespace h3

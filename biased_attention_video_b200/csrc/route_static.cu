@@ -17,13 +17,10 @@
 #include "h3attn.h"
 #include "kernels.cuh"
 
-namespace h3 {
-size_t route_smem_bytes(int d, int n_video);
-}
 
 namespace {
 
-// 32 MiB: pooled Q and K, 2 * H * n_video_blocks * d floats at most.
+// 32 MiB of routing scratch (two-part pooled centroids and the score matrix).
 constexpr size_t kStaticPooledFloats = size_t(8) << 20;
 constexpr int kMaxDevices = 64;
 
@@ -63,20 +60,15 @@ extern "C" int h3attn_route_static(const h3attn_plan* plan, const uint16_t* q, c
   if ((reinterpret_cast<uintptr_t>(q) & 15u) || (reinterpret_cast<uintptr_t>(k) & 15u) ||
       (reinterpret_cast<uintptr_t>(kv_sel) & 3u))
     return H3ATTN_EALIGN;
-  const size_t per_tensor = (size_t)plan->H * plan->n_video_blocks * plan->d;
-  if (2 * per_tensor > kStaticPooledFloats) return H3ATTN_EWORKSPACE;
+  const h3::RouteScratch need = h3::route_scratch_layout(plan->H, plan->d, plan->n_video_blocks);
+  if (need.total > kStaticPooledFloats * sizeof(float)) return H3ATTN_EWORKSPACE;
   if (h3::route_smem_bytes(plan->d, plan->n_video_blocks) > (size_t)227 * 1024) return H3ATTN_EUNSUPPORTED;
   int status = H3ATTN_OK;
   float* scratch = scratch_for_current_device(&status);
   if (scratch == nullptr) return status;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  float* qp = scratch;
-  float* kp = scratch + per_tensor;
-  if (h3::launch_pool(q, qp, k, kp, plan->H, plan->S, plan->d, plan->first_video_block, plan->n_video_blocks, st) !=
-      cudaSuccess)
-    return H3ATTN_ECUDA;
-  if (h3::launch_route(qp, kp, kv_sel, plan->H, plan->d, plan->n_video_blocks, plan->k, plan->first_video_block, st) !=
-      cudaSuccess)
+  if (h3::launch_route_pipeline(q, k, kv_sel, plan->H, plan->S, plan->d, plan->first_video_block,
+                                plan->n_video_blocks, plan->k, scratch, nullptr,
+                                static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return H3ATTN_ECUDA;
   return H3ATTN_OK;
 }

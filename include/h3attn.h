@@ -115,7 +115,9 @@ H3ATTN_API int h3attn_plan_init(h3attn_plan* plan, int H, int S, int d, int bloc
                      const uint8_t* seg_host);
 
 /* Bytes of device workspace a plan needs for h3attn_route and h3attn_forward
- * (status word, per-block key descriptors, pooled Q and K of the video blocks).
+ * (status word, per-block key descriptors, and the routing scratch: two-part
+ * bf16 pooled Q and K of the video blocks and the fp32 pooled-score matrix,
+ * about 0.9 GB at S = 116,883, H = 56, d = 128).
  * The caller allocates it once, zero-filled (the first 256 bytes hold the
  * status word that h3attn_check reads and clears). */
 H3ATTN_API size_t h3attn_workspace_bytes(const h3attn_plan* plan);
@@ -131,8 +133,11 @@ H3ATTN_API int h3attn_pool(const h3attn_plan* plan, const uint16_t* x, int first
 /* Routing (pool + pooled score + top-k).  For every head h and video query
  * block i (block first_video_block + i):
  *   kv_sel[h][i][0..k) = the k video key blocks j with the highest
- *   Qp[h][i].Kp[h][j] / sqrt(d) (fp32), ties to the lower block, listed as
- *   absolute block indices in ascending order.
+ *   Qp[h][i].Kp[h][j] / sqrt(d), ties to the lower block, listed as absolute
+ *   block indices in ascending order.  Qp, Kp are fp32 block means; the dot
+ *   products run on the tensor cores over two-part bf16 splits of them
+ *   (x = hi + lo, Qh.Kh + Qh.Kl + Ql.Kh accumulated in fp32: relative error
+ *   about 2^-16 per product).
  * q, k: bf16 [H][S][d] device; kv_sel: int32 [H][n_video_blocks][k] device.
  * ws: workspace of at least h3attn_workspace_bytes(plan) bytes. */
 H3ATTN_API int h3attn_route(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, int32_t* kv_sel,
@@ -143,10 +148,12 @@ H3ATTN_API int h3attn_route(const h3attn_plan* plan, const uint16_t* q, const ui
  * device memory when they route (a framework that owns all device memory
  * through its own pool, a loop that must not pay cudaMalloc's implicit
  * synchronisation, a host with a fixed memory budget).
- * Same result as h3attn_route.  Its scratch for the pooled Q and K is a fixed
- * 32 MiB array inside the library that every GPU loading the library holds
- * until the process exits; problems with 2 * H * n_video_blocks * d > 8,388,608
- * are rejected with H3ATTN_EWORKSPACE.  Every call overwrites all the scratch
+ * Same result as h3attn_route.  Its scratch (the two-part bf16 pooled
+ * centroids of Q and K and the fp32 score matrix) is a fixed 32 MiB array
+ * inside the library that every GPU loading the library holds until the
+ * process exits; problems needing more, i.e. with
+ * 12 * H * n_video_blocks * d + 16 * H * n_video_blocks * ceil(n_video_blocks / 4)
+ * bytes above about 32 MiB, are rejected with H3ATTN_EWORKSPACE.  Every call overwrites all the scratch
  * it reads, so nothing needs clearing between calls; calls that overlap on the
  * GPU (other streams, other threads) share the array and race.  The first call
  * on a device looks up the array's device address with that device current;
