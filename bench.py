@@ -85,6 +85,26 @@ def executed_mma_pairs(p, sel: np.ndarray | None) -> int:
     return int(total) * 128 * 128
 
 
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank runs its own independent call: the workload's seed shifted by the rank."""
+    return base_seed + rank
+
+
+def max_over_ranks(values, world: int, device="cpu"):
+    """Element-wise maximum of per-rank timings (all ranks take part; no-op for one rank)."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def whole_job_tflops(flops_per_call: float, calls_per_rank: int, world: int, ms: float) -> float:
+    """Aggregate throughput of all ranks: every rank did calls_per_rank calls in at most ms."""
+    return world * flops_per_call * calls_per_rank / (ms * 1e-3) / 1e12
+
+
 class ClockSampler:
     """nvidia-smi clock/throttle sampling while the timed region runs."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -219,7 +239,7 @@ def run_ours(args, rank, world, local_rank):
     if args.heads is not None:
         cfg = inputs.custom(args.heads, cfg.d, cfg.segments, cfg.seed, cluster_norm=cfg.cluster_norm,
                             penalty=cfg.penalty, sparsities=cfg.sparsities, name=f"{cfg.name} ({args.heads} heads)")
-    seed = cfg.seed + rank
+    seed = rank_seed(cfg.seed, rank)
     seg, times, _ = cfg.layout()
     H, S, d = cfg.H, cfg.S, cfg.d
     sparsity = cfg.sparsities[0]
@@ -323,17 +343,14 @@ def run_ours(args, rank, world, local_rank):
             raise RuntimeError("device status after e2e")
 
     # max over ranks
-    t = torch.tensor([ms, e2e_ms, fwd_ms, route_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms, e2e_ms, fwd_ms, route_ms = (float(x) for x in t.cpu())
+    ms, e2e_ms, fwd_ms, route_ms = max_over_ranks([ms, e2e_ms, fwd_ms, route_ms], world, dev)
 
     if rank != 0:
         return
     peaks, peak_kind = measured_peaks()
     ms_step = ms / args.steps
-    value = world * eff_flops * args.steps / (ms * 1e-3) / 1e12
-    e2e_value = world * eff_flops * args.steps / (e2e_ms * 1e-3) / 1e12
+    value = whole_job_tflops(eff_flops, args.steps, world, ms)
+    e2e_value = whole_job_tflops(eff_flops, args.steps, world, e2e_ms)
     attn_tflops = eff_flops / (fwd_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     route_bytes = 2 * H * p.n_video_blocks * 64 * d * 2  # Q and K video rows, read once by the pool
