@@ -37,6 +37,22 @@ WORKLOAD = "full combined: S=116883 (text 256|image-ref 1013|audio 810|guide 27x
            "H=56, d=128, bf16, block 64, sparsity 0.90 (k=180 of 1794 video KV blocks), default penalty"
 
 
+# DRAM bytes of one attn_kernel launch measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum of an
+# 8-head launch of this packing, profiles/attn_kernel_full_combined_H8.md), scaled by heads.  Valid only for
+# the kernel source it was taken from; reported as null once csrc/attn.cu changes.
+ATTN_TRAFFIC = {"source_sha256_prefix": "50fa7db55dbc960a", "bytes_per_head": (1.465091e9 + 0.239452e9) / 8}
+
+
+def attn_traffic_bytes(H: int):
+    import hashlib
+    path = os.path.join(ROOT, "biased_attention_video_b200", "csrc", "attn.cu")
+    with open(path, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()
+    if not digest.startswith(ATTN_TRAFFIC["source_sha256_prefix"]):
+        return None
+    return ATTN_TRAFFIC["bytes_per_head"] * H
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -365,7 +381,7 @@ def run_ours(args, rank, world, local_rank):
                    "executed_mma_tflop_per_call": 4 * d * mma_pairs / 1e12,
                    "route_ms": route_ms, "attention_ms": fwd_ms},
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
-                     "frac": attn_tflops / peak, "traffic": None,
+                     "frac": attn_tflops / peak, "traffic": attn_traffic_bytes(H),
                      "kernel": "attn_kernel (fused routed attention); achieved = effective FLOPs per launch / "
                                "CUDA-event time of the forward call (kv_desc prep + attention)",
                      "peak_source": f"{peak_kind} bf16_tflops_sustained"},
