@@ -16,17 +16,24 @@
 // Warp roles (320 threads; two CTAs per SM leave 96 registers per thread):
 //   warp 0      TMA producer: Q tile once, then K and V 128-key tiles
 //   warp 1      TMEM owner + single-thread tcgen05.mma issuer
-//   warps 2..9  softmax: two threads per query row (= TMEM lane), each owning
-//               half of the keys of a tile; warp w may only touch TMEM lanes
-//               [32 (w % 4), 32 (w % 4) + 32)
-// TMEM: S [0,128) fp32 scores; the bf16 probabilities P(j) are written over
-// its first 64 columns; O [128, 128 + d).
-// The softmax works on one 64-key half of a tile at a time and hands over P
-// half by half; the MMA warp issues PV(j, half 0) while the softmax works on
-// half 1.
-// MMA issue order S(0), PV(0,0), PV(0,1), S(1), ...: the tcgen05.mma ops of one
-// thread run in issue order, so S(j+1) never overwrites P(j) before PV(j) has
-// read it, and when the commit after S(j+1) fires, PV(j) is complete too.
+//   warps 2..9  softmax: two threads per query row (= TMEM lane); the thread
+//               of part p owns key block p of every tile (keys 64p..64p+63);
+//               warp w may only touch TMEM lanes [32 (w % 4), 32 (w % 4) + 32)
+//
+// TMEM: S [0,128) fp32 scores of the current tile; O [128, 128 + d).
+// Each softmax thread works on its 64 keys in two phases:
+//   phase 0, keys 0..47 of its block: bf16 probabilities go back into TMEM
+//            over the block's first 24 score columns (TS-form PV);
+//   phase 1, keys 48..63: probabilities go to an 8 KB shared-memory tile
+//            (SS-form PV).
+// Before handing phase 0 over, each thread has already read its phase-1
+// scores, so the whole S region is free once PV(j, phase 0) has read its P:
+// the MMA warp issues S(j+1) right behind PV(j, phase 0), and the next tile's
+// scores are computed while the softmax still works on phase 1 of this one.
+// MMA issue order: S(0) | PV(0,0) S(1) PV(0,1) | PV(1,0) S(2) PV(1,1) | ...
+// The tcgen05.mma ops of one thread run in issue order, so S(j+1) never
+// overwrites P(j, phase 0) before PV(j, phase 0) has read it, and when the
+// commit after S(j+1) fires, PV(j, phase 0) is complete too.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -41,6 +48,7 @@ namespace {
 constexpr int kThreads = 320;
 constexpr int kTileRows = 128;  // query rows per CTA
 constexpr int kTileKeys = 128;  // keys per KV tile
+constexpr int kPhase0Keys = 48;  // keys per block whose P stays in TMEM
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kTmemO = 128;  // O column offset
 constexpr float kLn2 = 0.6931471805599453f;
@@ -64,9 +72,13 @@ struct Layout {
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kTileBytes;
   static constexpr int kV = kK + kTileBytes;
-  static constexpr int kBars = kV + kTileBytes;
-  // barriers: q_full, k_full, k_empty, v_full, v_empty, s_full, p_full[2], o_half0, o_final, drain, xchg[4]
-  static constexpr int kNumBars = 15;
+  // phase-1 probabilities: two K-major 32-byte-swizzled operands (one per key
+  // block of the tile), 128 rows x 16 keys each
+  static constexpr int kPh1 = kV + kTileBytes;
+  static constexpr int kPh1StepBytes = kTileRows * 32;
+  static constexpr int kBars = kPh1 + 2 * kPh1StepBytes;
+  // q_full, k_full, k_empty, v_full, v_empty, s_full, p_full[2], o_half0, o_done, o_final, drain, xchg[4]
+  static constexpr int kNumBars = 16;
   static constexpr int kMisc = kBars + kNumBars * 8;  // tmem base, abort flag, n_entries
   static constexpr int kRed = kMisc + 16;             // partial row maxima / sums: float [2][2][128]
   static constexpr int kBitmaps = kRed + 2 * 2 * 128 * 4;
@@ -77,17 +89,21 @@ struct Layout {
 };
 
 struct Bars {
-  uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *o_half0, *o_final, *drain, *xchg;
+  uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *o_half0, *o_done, *o_final, *drain,
+      *xchg;
 };
 
-// p_full[h]: P of half h of the current tile is in TMEM (one completion per
-// tile each, so a waiter is never more than one phase behind).
+// p_full[ph]: P of phase ph of the current tile is in place (one completion
+// per tile each, so a waiter is never more than one phase behind).
+// o_half0 / o_done: PV(j, phase 0) / PV(j, phase 1) complete.  The softmax
+// waits for both on every tile (o_done(j-1) in phase 0 of tile j, o_half0(j)
+// in phase 1), so its parity never falls behind either.
 // xchg[q]: the two softmax warps of TMEM lane quarter q have written their
 // partial row values (64 arrivals per exchange; neither warp can run more than
 // one exchange ahead of the other).
 __device__ __forceinline__ Bars carve_bars(uint8_t* base) {
   uint64_t* b = reinterpret_cast<uint64_t*>(base);
-  return Bars{b, b + 1, b + 2, b + 3, b + 4, b + 5, b + 6, b + 8, b + 9, b + 10, b + 11};
+  return Bars{b, b + 1, b + 2, b + 3, b + 4, b + 5, b + 6, b + 8, b + 9, b + 10, b + 11, b + 12};
 }
 
 // Bounded wait with CTA-wide abort.  On give-up: raise the CTA abort flag and
@@ -135,6 +151,100 @@ __device__ __forceinline__ float block_penalty_log2(float tq, float tk, const At
   return fminf(p.strength_log2 * ex * ex, p.cap_log2);
 }
 
+// How a thread treats its key block in the current tile.
+struct BlockMode {
+  int mode;     // 0 skip (not attended by this row), 1 plain, 2 constant penalty, 3 per-key penalty
+  int nv;       // valid keys of the block
+  int key0;     // first key (sequence row) of the block
+  float cpen;   // constant penalty (mode 2), log2 units
+};
+
+// Probabilities of 16 keys [c0, c0 + 16) of the thread's block, given the row
+// max m (log2 units), as 8 bf16 pairs; returns their fp32 sum.
+__device__ __forceinline__ float probs16(const float* s, const BlockMode& bm, int c0, float m, float scale,
+                                         float tq, const AttnParams& p, uint32_t* pk) {
+  float lt = 0.0f;
+  if (bm.mode == 0) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) pk[i] = 0u;
+  } else if (bm.mode == 3) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float pp[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int col = c0 + 2 * i + e;
+        float pen_k = 0.0f;
+        if (col < bm.nv && p.seg[bm.key0 + col] == kSegGuide)
+          pen_k = block_penalty_log2(tq, p.times[bm.key0 + col], p);
+        pp[e] = col < bm.nv ? ex2(fmaf(s[2 * i + e], scale, -(m + pen_k))) : 0.0f;
+      }
+      lt += pp[0] + pp[1];
+      pk[i] = pack_bf16(pp[0], pp[1]);
+    }
+  } else if (bm.nv >= c0 + 16) {
+    // pairs in packed fp32: scale and offset by one f32x2 FMA; one pair in
+    // four takes 2^x on the FMA pipe, the rest on MUFU
+    const float off = -(m + bm.cpen);
+    const uint64_t scale2 = f2_pack(scale, scale), off2 = f2_pack(off, off);
+    uint64_t acc2[2] = {f2_pack(0.0f, 0.0f), f2_pack(0.0f, 0.0f)};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint64_t x2 = f2_fma(f2_pack(s[2 * i], s[2 * i + 1]), scale2, off2);
+      uint64_t p2;
+      if ((i & 3) == 3) {
+        p2 = ex2_poly2(x2);
+      } else {
+        float a, b;
+        f2_unpack(x2, a, b);
+        p2 = f2_pack(ex2(a), ex2(b));
+      }
+      acc2[i & 1] = f2_add(acc2[i & 1], p2);
+      float p0, p1;
+      f2_unpack(p2, p0, p1);
+      pk[i] = pack_bf16(p0, p1);
+    }
+    float a0, a1, b0, b1;
+    f2_unpack(acc2[0], a0, a1);
+    f2_unpack(acc2[1], b0, b1);
+    lt = (a0 + a1) + (b0 + b1);
+  } else {
+    const float off = -(m + bm.cpen);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int col = c0 + 2 * i;
+      const float p0 = col < bm.nv ? ex2(fmaf(s[2 * i], scale, off)) : 0.0f;
+      const float p1 = col + 1 < bm.nv ? ex2(fmaf(s[2 * i + 1], scale, off)) : 0.0f;
+      lt += p0 + p1;
+      pk[i] = pack_bf16(p0, p1);
+    }
+  }
+  return lt;
+}
+
+// Maximum over the valid keys [c0, c0 + N) of the thread's block (-inf if none).
+template <int N>
+__device__ __forceinline__ float part_max(const float* s, const BlockMode& bm, int c0) {
+  float pmax = -INFINITY;
+  if (bm.mode != 0) {
+    if (bm.nv >= c0 + N) {
+      float mp[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) mp[a] = fmaxf(s[a], s[a + 4]);
+#pragma unroll
+      for (int i = 8; i < N; i += 8)
+#pragma unroll
+        for (int a = 0; a < 4; ++a) mp[a] = max3f(mp[a], s[i + a], s[i + 4 + a]);
+      pmax = fmaxf(max3f(mp[0], mp[1], mp[2]), mp[3]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < N; ++i)
+        if (c0 + i < bm.nv) pmax = fmaxf(pmax, s[i]);
+    }
+  }
+  return pmax;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -180,6 +290,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     mbar_init(bars.p_full, 8);
     mbar_init(bars.p_full + 1, 8);
     mbar_init(bars.o_half0, 1);
+    mbar_init(bars.o_done, 1);
     mbar_init(bars.o_final, 1);
     mbar_init(bars.drain, 1);
     for (int q = 0; q < 4; ++q) mbar_init(bars.xchg + q, 64);
@@ -270,9 +381,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int oob_row = p.n_blocks * 64;  // a whole block past S: zero-filled by TMA
       for (int j = 0; j < n_tiles; ++j) {
         const uint32_t ph = (uint32_t)j & 1u;
-        const int e0 = (int)(list[2 * j] & 0x3FFFu);
-        const int e1 = (2 * j + 1 < n_entries) ? (int)(list[2 * j + 1] & 0x3FFFu) : -1;
-        const int r0 = e0 * 64, r1 = e1 >= 0 ? e1 * 64 : oob_row;
+        const int r0 = (int)(list[2 * j] & 0x3FFFu) * 64;
+        const int r1 = (2 * j + 1 < n_entries) ? (int)(list[2 * j + 1] & 0x3FFFu) * 64 : oob_row;
         if (!wait_bar(bars.k_empty, ph ^ 1u, p, abort_flag)) break;
         mbar_arrive_expect_tx(bars.k_full, L::kTileBytes);
 #pragma unroll
@@ -301,6 +411,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint32_t q_addr = smem_u32(smem + L::kQ);
       const uint32_t k_addr = smem_u32(smem + L::kK);
       const uint32_t v_addr = smem_u32(smem + L::kV);
+      const uint32_t ph1_addr = smem_u32(smem + L::kPh1);
       const uint32_t tmem_s = tmem_base;
       const uint32_t tmem_o = tmem_base + kTmemO;
       auto issue_s = [&](int j) -> bool {
@@ -321,26 +432,40 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (ok && n_tiles > 0) ok = issue_s(0);
       for (int j = 0; ok && j < n_tiles; ++j) {
         const uint32_t ph = (uint32_t)j & 1u;
-        if (!wait_bar(bars.v_full, ph, p, abort_flag)) {
+        if (!wait_bar(bars.v_full, ph, p, abort_flag) || !wait_bar(bars.p_full, ph, p, abort_flag)) {
           ok = false;
           break;
         }
+        tc_fence_after();
+        // PV(j, phase 0): keys 16c..16c+15 of block b (c < 3) = V rows 64b+16c..,
+        // P in TMEM columns 64b + 8c (B = V tile, MN-major: 16 keys per step)
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          if (!wait_bar(bars.p_full + hh, ph, p, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+        for (int b = 0; b < 2; ++b)
 #pragma unroll
-          for (int kk = hh * 4; kk < hh * 4 + 4; ++kk) {
-            // B = V tile, MN-major: 16 keys per step = two 8-row swizzle groups
-            const uint64_t bdesc = sw128_desc(v_addr + kk * 2048, L::kHalfBytes, 1024);
-            umma_ts(tmem_o, tmem_s + kk * 8, bdesc, kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
+          for (int c = 0; c < kPhase0Keys / 16; ++c) {
+            const uint64_t bdesc = sw128_desc(v_addr + (4 * b + c) * 2048, L::kHalfBytes, 1024);
+            umma_ts(tmem_o, tmem_s + 64 * b + 8 * c, bdesc, kIdescO, (j > 0 || b > 0 || c > 0) ? 1u : 0u);
           }
-          umma_commit(hh == 0 ? bars.o_half0 : bars.v_empty);
+        umma_commit(bars.o_half0);
+        // S(j+1): every thread has read its phase-1 scores before p_full[0]
+        if (j + 1 < n_tiles && !issue_s(j + 1)) {
+          ok = false;
+          break;
         }
-        if (ok && j + 1 < n_tiles) ok = issue_s(j + 1);
+        if (!wait_bar(bars.p_full + 1, ph, p, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // PV(j, phase 1): keys 48..63 of block b, P from shared memory
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          const uint64_t adesc = sw32_kmajor_desc(ph1_addr + b * L::kPh1StepBytes);
+          const uint64_t bdesc = sw128_desc(v_addr + (4 * b + 3) * 2048, L::kHalfBytes, 1024);
+          umma_ss(tmem_o, adesc, bdesc, kIdescO, 1u);
+        }
+        umma_commit(bars.v_empty);
+        umma_commit(bars.o_done);
       }
       umma_commit(bars.o_final);
       // drain: all issued MMAs complete before TMEM is released
@@ -350,11 +475,10 @@ __global__ void __launch_bounds__(kThreads, 2)
   } else {
     // ------------------------------------------------------------ softmax
     // Two threads per query row: warp w handles TMEM lanes [32 (w % 4), +32)
-    // and, inside every 64-key half, the 32 keys [32 part, 32 part + 32) with
-    // part = (w - 2) / 4.  The two threads of a row exchange their partial
-    // maxima through shared memory (one named barrier per lane quarter), so
-    // both apply the same running max; each rescales and finally normalises
-    // its half of O's columns.
+    // and key block part = (w - 2) / 4 of every tile.  The two threads of a
+    // row exchange their partial maxima through shared memory (an mbarrier per
+    // lane quarter), so both apply the same running max; each rescales and
+    // finally normalises its half of O's columns.
     // tcgen05.ld/st are warp-collective (.sync.aligned): every branch that
     // guards one is made warp-uniform with __all_sync / __any_sync.
     constexpr int kOCols = D / 2;  // O columns per thread
@@ -362,11 +486,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int part = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;  // row within the tile == TMEM lane
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-    const uint32_t t_s = tmem_base + lane_addr;
+    const uint32_t t_s = tmem_base + lane_addr + (uint32_t)(64 * part);  // this thread's block of S
     const uint32_t t_o = tmem_base + lane_addr + kTmemO + (uint32_t)(part * kOCols);
     uint64_t* xbar = bars.xchg + quarter;
     uint32_t n_xchg = 0;  // exchanges done (phase parity of xbar)
     float* red = reinterpret_cast<float*>(smem + L::kRed);  // [2 slots][2 parts][128 rows]
+    // phase-1 probabilities of this row: 32 bytes at row r of this part's operand
+    uint8_t* ph1_row = smem + L::kPh1 + part * L::kPh1StepBytes + r * 32;
+    const uint32_t ph1_swz = (uint32_t)((r >> 2) & 1) << 4;  // 32-byte swizzle: bit 4 ^= bit 7
     const int my_bit = 14 + (r >> 6);  // list bit of this row's query block
     const int qrow = qtile * kTileRows + r;
     const bool row_valid = qrow < p.S;
@@ -376,188 +503,157 @@ __global__ void __launch_bounds__(kThreads, 2)
     float m = -INFINITY;  // running max, log2 units (upper bound of the true max)
     float l = 0.0f;       // partial row sum over this thread's keys
     bool ok = true;
-    for (int j = 0; ok && j < n_tiles; ++j) {
-      // this tile's two key blocks and their descriptors, fetched before the
-      // wait so the loads overlap it
-      uint32_t ents[2];
-      uint2 kds[2];
+
+    // Combine this thread's partial max with its partner's (slot `slot`: a
+    // slot is rewritten only after the next exchange's barrier, which both
+    // threads pass after reading it).  Returns false on give-up.
+    auto exchange_max = [&](float pmax, int slot, float& mx) -> bool {
+      red[(slot * 2 + part) * 128 + r] = pmax;
+      mbar_arrive(xbar);
+      const bool gotx = wait_bar(xbar, n_xchg & 1u, p, abort_flag);
+      ++n_xchg;
+      if (!__all_sync(kFull, gotx)) return false;
+      mx = fmaxf(pmax, red[(slot * 2 + (part ^ 1)) * 128 + r]) * scale;
+      return true;
+    };
+    // O *= alpha for this thread's O columns (warp-uniform call)
+    auto rescale_o = [&](float alpha) {
+#pragma unroll 1
+      for (int c = 0; c < kOCols / 16; ++c) {
+        uint32_t tmp[16];
+        __syncwarp();
+        tmem_ld16(t_o + c * 16, tmp);
+        tmem_wait_ld();
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int idx = 2 * j + hh;
-        ents[hh] = idx < n_entries ? (uint32_t)list[idx] : 0u;
-        kds[hh] = ((ents[hh] >> my_bit) & 1u) ? __ldg(p.kv_desc + (ents[hh] & 0x3FFFu)) : make_uint2(0u, 0u);
+        for (int i = 0; i < 16; ++i) tmp[i] = __float_as_uint(__uint_as_float(tmp[i]) * alpha);
+        tmem_st16(t_o + c * 16, tmp);
       }
-      const bool got = wait_bar(bars.s_full, (uint32_t)j & 1u, p, abort_flag);
-      if (!__all_sync(kFull, got)) {
+    };
+
+    for (int j = 0; ok && j < n_tiles; ++j) {
+      const uint32_t ph = (uint32_t)j & 1u;
+      // this thread's key block and its descriptor, fetched before the wait
+      const int idx = 2 * j + part;
+      const uint32_t ent = idx < n_entries ? (uint32_t)list[idx] : 0u;
+      const bool attended = idx < n_entries && ((ent >> my_bit) & 1u);
+      const uint2 kd = attended ? __ldg(p.kv_desc + (ent & 0x3FFFu)) : make_uint2(0u, 0u);
+      BlockMode bm{0, 0, (int)(ent & 0x3FFFu) * 64, 0.0f};
+      if (attended) {
+        bm.nv = (int)(kd.x & 0xFFu);
+        const int kind = (int)((kd.x >> 8) & 3u);
+        bm.mode = 1;
+        if (pen_row && kind == 1) {
+          bm.cpen = block_penalty_log2(tq, __uint_as_float(kd.y), p);
+          bm.mode = 2;
+        } else if (pen_row && kind == 2) {
+          bm.mode = 3;
+        }
+      }
+      if (!__all_sync(kFull, wait_bar(bars.s_full, ph, p, abort_flag))) {
         ok = false;
         break;
       }
       tc_fence_after();
+
+      // ---------------- phase 0: keys 0..47 of the block, P back into TMEM
+      float sv[kPhase0Keys];
+      {
+        uint32_t t32[32], t16[16];
+        __syncwarp();
+        tmem_ld32(t_s, t32);
+        tmem_ld16(t_s + 32, t16);
+        tmem_wait_ld();
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        // this half: 0 skip, 1 plain, 2 constant penalty, 3 per-key penalty
-        int mode = 0, nv = 0, kblock = 0;
-        float cpen = 0.0f;
-        const int idx = 2 * j + hh;
-        if (idx < n_entries) {
-          const uint32_t ent = ents[hh];
-          kblock = (int)(ent & 0x3FFFu);
-          if ((ent >> my_bit) & 1u) {
-            const uint2 kd = kds[hh];
-            nv = (int)(kd.x & 0xFFu);
-            const int kind = (int)((kd.x >> 8) & 3u);
-            mode = 1;
-            if (pen_row && kind == 1) {
-              cpen = block_penalty_log2(tq, __uint_as_float(kd.y), p);
-              mode = 2;
-            } else if (pen_row && kind == 2) {
-              mode = 3;
-            }
-          }
-        }
-        const int col0 = part * 32;  // first key of this thread inside the half
-        float sv[32];
-        {
-          uint32_t tmp[32];
-          __syncwarp();
-          tmem_ld32(t_s + hh * 64 + col0, tmp);
-          tmem_wait_ld();
+        for (int i = 0; i < 32; ++i) sv[i] = __uint_as_float(t32[i]);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) sv[i] = __uint_as_float(tmp[i]);
-        }
-        float pmax = -INFINITY;
-        if (mode != 0) {
-          if (nv == 64) {
-            float mp[4];
+        for (int i = 0; i < 16; ++i) sv[32 + i] = __uint_as_float(t16[i]);
+      }
+      float mx;
+      if (!exchange_max(part_max<kPhase0Keys>(sv, bm, 0), 0, mx)) {
+        ok = false;
+        break;
+      }
+      // Conditional rescale: the running max only moves when it grows by more
+      // than 2^8; below that the stale max keeps every probability <= 256.
+      bool grow = mx > m + kRescaleThreshold;
+      bool o_rescale = grow && m > -INFINITY;
+      float m_old = m;
+      if (grow) m = mx;
+      float lt = 0.0f;
 #pragma unroll
-            for (int a = 0; a < 4; ++a) mp[a] = fmaxf(sv[a], sv[a + 4]);
+      for (int g = 0; g < kPhase0Keys / 16; ++g) {
+        uint32_t pk[8];
+        lt += probs16(sv + 16 * g, bm, 16 * g, m, scale, tq, p, pk);
+        __syncwarp();
+        tmem_st8(t_s + 8 * g, pk);  // P of keys 16g..16g+15 over score columns 8g..8g+7
+      }
+      // phase-1 scores: read now, so that S(j+1) may overwrite the S region
+      // as soon as PV(j, phase 0) has consumed P
+      float sv1[16];
+      {
+        uint32_t t16[16];
+        __syncwarp();
+        tmem_ld16(t_s + kPhase0Keys, t16);
+        tmem_wait_ld();
 #pragma unroll
-            for (int i = 8; i < 32; i += 8)
-#pragma unroll
-              for (int a = 0; a < 4; ++a) mp[a] = max3f(mp[a], sv[i + a], sv[i + 4 + a]);
-            pmax = fmaxf(max3f(mp[0], mp[1], mp[2]), mp[3]);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (col0 + i < nv) pmax = fmaxf(pmax, sv[i]);
-          }
-        }
-        // combine the two partial maxima of the row (slot hh: a slot is
-        // rewritten only after the next exchange's barrier, which both threads
-        // pass after reading it)
-        red[(hh * 2 + part) * 128 + r] = pmax;
-        mbar_arrive(xbar);
-        const bool gotx = wait_bar(xbar, n_xchg & 1u, p, abort_flag);
-        ++n_xchg;
-        if (!__all_sync(kFull, gotx)) {
+        for (int i = 0; i < 16; ++i) sv1[i] = __uint_as_float(t16[i]);
+      }
+      // O is stable once PV(j-1, phase 1) has completed (waited on every tile)
+      if (j > 0) {
+        if (!__all_sync(kFull, wait_bar(bars.o_done, ph ^ 1u, p, abort_flag))) {
           ok = false;
           break;
         }
-        const float mx = fmaxf(pmax, red[(hh * 2 + (part ^ 1)) * 128 + r]) * scale;
-        // Conditional rescale: the running max only moves when it grows by
-        // more than 2^8; below that the stale max keeps every probability <= 256.
-        const bool grow = mx > m + kRescaleThreshold;
-        const bool o_rescale = grow && m > -INFINITY;
-        const float m_old = m;
-        if (grow) m = mx;
-        // probabilities of this thread's 32 keys -> bf16 pairs into P columns
-        // [32 hh + 16 part, +16) (P(j) overwrites the first 64 columns of S)
-        float lt = 0.0f;
-        uint32_t packed[16];
-        if (mode == 0) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) packed[i] = 0u;
-        } else if (mode == 3) {
-          const int key0 = kblock * 64 + col0;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float pp[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int col = col0 + 2 * i + e;
-              float pen_k = 0.0f;
-              if (col < nv && p.seg[key0 + 2 * i + e] == kSegGuide)
-                pen_k = block_penalty_log2(tq, p.times[key0 + 2 * i + e], p);
-              pp[e] = col < nv ? ex2(fmaf(sv[2 * i + e], scale, -(m + pen_k))) : 0.0f;
-            }
-            lt += pp[0] + pp[1];
-            packed[i] = pack_bf16(pp[0], pp[1]);
-          }
-        } else if (nv == 64) {
-          // pairs in packed fp32: scale and offset by one f32x2 FMA; one pair
-          // in four takes 2^x on the FMA pipe, the rest on MUFU
-          const float off = -(m + cpen);
-          const uint64_t scale2 = f2_pack(scale, scale), off2 = f2_pack(off, off);
-          uint64_t acc2[2] = {f2_pack(0.0f, 0.0f), f2_pack(0.0f, 0.0f)};
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const uint64_t x2 = f2_fma(f2_pack(sv[2 * i], sv[2 * i + 1]), scale2, off2);
-            uint64_t p2;
-            if ((i & 3) == 3) {
-              p2 = ex2_poly2(x2);
-            } else {
-              float a, b;
-              f2_unpack(x2, a, b);
-              p2 = f2_pack(ex2(a), ex2(b));
-            }
-            acc2[i & 1] = f2_add(acc2[i & 1], p2);
-            float p0, p1;
-            f2_unpack(p2, p0, p1);
-            packed[i] = pack_bf16(p0, p1);
-          }
-          float a0, a1, b0, b1;
-          f2_unpack(acc2[0], a0, a1);
-          f2_unpack(acc2[1], b0, b1);
-          lt = (a0 + a1) + (b0 + b1);
-        } else {
-          const float off = -(m + cpen);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int col = col0 + 2 * i;
-            const float p0 = col < nv ? ex2(fmaf(sv[2 * i], scale, off)) : 0.0f;
-            const float p1 = col + 1 < nv ? ex2(fmaf(sv[2 * i + 1], scale, off)) : 0.0f;
-            lt += p0 + p1;
-            packed[i] = pack_bf16(p0, p1);
-          }
-        }
-        __syncwarp();
-        tmem_st16(t_s + hh * 32 + part * 16, packed);
-        // O rescale (rare), after the scores are dead to keep registers low
-        float alpha = 1.0f;
-        if (__any_sync(kFull, o_rescale)) {
-          // Half 0: O is stable (PV(j-1) completed before S(j) did).  Half 1:
-          // wait for PV(j, half 0), issued once P of half 0 was handed over.
-          if (hh == 1) {
-            const bool got2 = wait_bar(bars.o_half0, (uint32_t)j & 1u, p, abort_flag);
-            if (!__all_sync(kFull, got2)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-          }
-          alpha = o_rescale ? ex2(m_old - m) : 1.0f;
-#pragma unroll
-          for (int c = 0; c < kOCols / 32; ++c) {
-            uint32_t tmp[32];
-            __syncwarp();
-            tmem_ld32(t_o + c * 32, tmp);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) tmp[i] = __float_as_uint(__uint_as_float(tmp[i]) * alpha);
-            tmem_st32(t_o + c * 32, tmp);
-          }
-        }
-        l = l * alpha + lt;
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bars.p_full + hh);  // one arrival per softmax warp
+        tc_fence_after();
       }
+      float alpha = 1.0f;
+      if (__any_sync(kFull, o_rescale)) {
+        alpha = o_rescale ? ex2(m_old - m) : 1.0f;
+        rescale_o(alpha);
+      }
+      l = l * alpha + lt;
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.p_full);  // one arrival per softmax warp
+
+      // ---------------- phase 1: keys 48..63, P to shared memory
+      if (!exchange_max(part_max<16>(sv1, bm, kPhase0Keys), 1, mx)) {
+        ok = false;
+        break;
+      }
+      grow = mx > m + kRescaleThreshold;
+      o_rescale = grow && m > -INFINITY;
+      m_old = m;
+      if (grow) m = mx;
+      {
+        uint32_t pk[8];
+        lt = probs16(sv1, bm, kPhase0Keys, m, scale, tq, p, pk);
+        // PV(j-1, phase 1) read the previous contents: complete (o_done above)
+        *reinterpret_cast<uint4*>(ph1_row + (0u ^ ph1_swz)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(ph1_row + (16u ^ ph1_swz)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      }
+      fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor core
+      alpha = 1.0f;
+      if (!__all_sync(kFull, wait_bar(bars.o_half0, ph, p, abort_flag))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (__any_sync(kFull, o_rescale)) {
+        alpha = o_rescale ? ex2(m_old - m) : 1.0f;
+        rescale_o(alpha);
+        tmem_wait_st();
+      }
+      l = l * alpha + lt;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.p_full + 1);
     }
     // ---------------------------------------------------------- epilogue
     bool fin = __all_sync(kFull, ok) && n_tiles > 0;
     // total row sum: slot 0 is free here (its last reader passed the barrier
-    // of the final half-1 exchange before this thread did)
+    // of the final phase-1 exchange before this thread did)
     if (fin) {
       red[part * 128 + r] = l;
       mbar_arrive(xbar);
