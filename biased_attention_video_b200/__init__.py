@@ -26,7 +26,7 @@ SEG_TEXT, SEG_IMAGE_REF, SEG_AUDIO, SEG_GUIDE, SEG_OUTPUT = 0, 1, 2, 3, 4
 EXPORTS = ("h3attn_plan_init", "h3attn_workspace_bytes", "h3attn_pool", "h3attn_route", "h3attn_route_static",
            "h3attn_forward",
            "h3attn_dense_workspace_bytes", "h3attn_dense_biased", "h3attn_check", "h3attn_selftest_timeout",
-           "h3attn_selftest_exp2", "h3attn_strerror")
+           "h3attn_strerror")
 
 
 class H3Error(RuntimeError):
@@ -89,8 +89,6 @@ def lib():
         L.h3attn_check.restype = ctypes.c_int
         L.h3attn_selftest_timeout.argtypes = [_P, ctypes.c_uint32, _P]
         L.h3attn_selftest_timeout.restype = ctypes.c_int
-        L.h3attn_selftest_exp2.argtypes = [_P, _P, ctypes.c_int, _P]
-        L.h3attn_selftest_exp2.restype = ctypes.c_int
         L.h3attn_strerror.argtypes = [ctypes.c_int]
         L.h3attn_strerror.restype = ctypes.c_char_p
         _lib = L
@@ -219,12 +217,3 @@ def check(ws: torch.Tensor, stream=None) -> int:
 
 def selftest_timeout(ws: torch.Tensor, polls: int, stream=None) -> None:
     _raise(lib().h3attn_selftest_timeout(ws.data_ptr(), polls, _stream(stream)), "selftest_timeout")
-
-
-def selftest_exp2(x: torch.Tensor, stream=None) -> torch.Tensor:
-    """2^x through the attention softmax's FMA-pipe exponential (float32 CUDA, even length)."""
-    if not (x.is_cuda and x.dtype == torch.float32 and x.is_contiguous()):
-        raise ValueError("x must be contiguous CUDA float32")
-    y = torch.empty_like(x)
-    _raise(lib().h3attn_selftest_exp2(x.data_ptr(), y.data_ptr(), x.numel(), _stream(stream)), "selftest_exp2")
-    return y

@@ -24,14 +24,24 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 struct WsLayout {
-  size_t desc, route, total;
+  size_t desc, gtime, slow, route, total;
 };
 
-// status word | per-key-block descriptors | routing scratch
+// Attention scratch after the status word: per-key-block descriptors, per-key
+// guide times (a guide key's time, NaN for every other key; padded to whole
+// blocks), and the bitmap of key blocks that need per-key treatment.
+size_t attn_scratch_bytes(int n_blocks) {
+  return align_up((size_t)n_blocks * sizeof(uint4)) + align_up((size_t)n_blocks * h3::kBlock * sizeof(float)) +
+         align_up((size_t)(n_blocks + 31) / 32 * sizeof(uint32_t));
+}
+
+// status word | per-key-block descriptors | per-key guide times | routing scratch
 WsLayout ws_layout(int H, int d, int n_blocks, int n_video) {
   WsLayout w;
   w.desc = kStatusBytes;
-  w.route = w.desc + align_up((size_t)n_blocks * sizeof(uint2));
+  w.gtime = w.desc + align_up((size_t)n_blocks * sizeof(uint4));
+  w.slow = w.gtime + align_up((size_t)n_blocks * h3::kBlock * sizeof(float));
+  w.route = kStatusBytes + attn_scratch_bytes(n_blocks);
   w.total = w.route + (n_video > 0 ? h3::route_scratch_layout(H, d, n_video).total : 0);
   return w;
 }
@@ -102,7 +112,10 @@ int forward_impl(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, 
   p.lse = lse;
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   p.status = reinterpret_cast<int*>(wsb);
-  p.kv_desc = reinterpret_cast<const uint2*>(wsb + kStatusBytes);
+  const WsLayout wl = ws_layout(plan->H, plan->d, plan->n_blocks, 0);
+  p.kv_desc = reinterpret_cast<const uint4*>(wsb + wl.desc);
+  p.gtime = reinterpret_cast<const float*>(wsb + wl.gtime);
+  p.slow_blocks = reinterpret_cast<const uint32_t*>(wsb + wl.slow);
   p.pen_on = pen_on ? 1 : 0;
   const float log2e = 1.4426950408889634f;
   p.scale_log2 = log2e / std::sqrt((float)plan->d);
@@ -120,8 +133,9 @@ int forward_impl(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, 
   if (!make_map(&tq, q, plan->H, plan->S, plan->d) || !make_map(&tk, k, plan->H, plan->S, plan->d) ||
       !make_map(&tv, v, plan->H, plan->S, plan->d))
     return H3ATTN_ECUDA;
-  if (h3::launch_kv_desc(seg, pen_on ? times : nullptr, plan->S, plan->n_blocks,
-                         reinterpret_cast<uint2*>(wsb + kStatusBytes), stream) != cudaSuccess)
+  if (h3::launch_kv_desc(seg, pen_on ? times : nullptr, plan->S, plan->n_blocks, reinterpret_cast<uint4*>(wsb + wl.desc),
+                         reinterpret_cast<float*>(wsb + wl.gtime), reinterpret_cast<uint32_t*>(wsb + wl.slow),
+                         stream) != cudaSuccess)
     return H3ATTN_ECUDA;
   if (h3::launch_attn(tq, tk, tv, p, n_qtiles * plan->H, stream) != cudaSuccess) return H3ATTN_ECUDA;
   return H3ATTN_OK;
@@ -219,7 +233,7 @@ int h3attn_forward(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k
                    const uint8_t* seg, const float* times, const h3attn_penalty* pen, const int32_t* kv_sel,
                    uint16_t* o, float* lse, void* ws, size_t ws_bytes, void* stream) {
   if (!plan_ok(plan)) return H3ATTN_EINVAL;
-  const size_t need = kStatusBytes + align_up((size_t)plan->n_blocks * sizeof(uint2));
+  const size_t need = kStatusBytes + attn_scratch_bytes(plan->n_blocks);
   if (kv_sel != nullptr && (reinterpret_cast<uintptr_t>(kv_sel) & 3u)) return H3ATTN_EALIGN;
   return forward_impl(plan, q, k, v, seg, times, pen, kv_sel, o, lse, ws, ws_bytes, need,
                       static_cast<cudaStream_t>(stream));
@@ -228,7 +242,7 @@ int h3attn_forward(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k
 size_t h3attn_dense_workspace_bytes(int S) {
   if (S <= 0) return 0;
   const int n_blocks = (S + h3::kBlock - 1) / h3::kBlock;
-  return kStatusBytes + align_up((size_t)n_blocks * sizeof(uint2));
+  return kStatusBytes + attn_scratch_bytes(n_blocks);
 }
 
 int h3attn_dense_biased(int H, int S, int d, const uint16_t* q, const uint16_t* k, const uint16_t* v,
@@ -269,13 +283,6 @@ int h3attn_selftest_timeout(void* ws, uint32_t polls, void* stream) {
   if (ws == nullptr || !aligned16(ws)) return H3ATTN_EINVAL;
   if (h3::launch_selftest_timeout(static_cast<int*>(ws), polls, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return H3ATTN_ECUDA;
-  return H3ATTN_OK;
-}
-
-int h3attn_selftest_exp2(const float* x, float* y, int n, void* stream) {
-  if (x == nullptr || y == nullptr || n < 0 || (n & 1)) return H3ATTN_EINVAL;
-  if ((reinterpret_cast<uintptr_t>(x) & 7u) || (reinterpret_cast<uintptr_t>(y) & 7u)) return H3ATTN_EALIGN;
-  if (h3::launch_selftest_exp2(x, y, n / 2, static_cast<cudaStream_t>(stream)) != cudaSuccess) return H3ATTN_ECUDA;
   return H3ATTN_OK;
 }
 

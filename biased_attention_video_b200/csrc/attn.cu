@@ -37,6 +37,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
+#include <type_traits>
 
 #include "fastmath.cuh"
 #include "kernels.cuh"
@@ -79,7 +80,7 @@ struct Layout {
   static constexpr int kBars = kPh1 + 2 * kPh1StepBytes;
   // q_full, k_full, k_empty, v_full, v_empty, s_full, p_full[2], o_half0, o_done, o_final, drain, xchg[4]
   static constexpr int kNumBars = 16;
-  static constexpr int kMisc = kBars + kNumBars * 8;  // tmem base, abort flag, n_entries
+  static constexpr int kMisc = kBars + kNumBars * 8;  // tmem base, abort flag, n_entries, n_fast
   static constexpr int kRed = kMisc + 16;             // partial row maxima / sums: float [2][2][128]
   static constexpr int kBitmaps = kRed + 2 * 2 * 128 * 4;
   static int host_bytes(int n_blocks) {
@@ -151,75 +152,95 @@ __device__ __forceinline__ float block_penalty_log2(float tq, float tk, const At
   return fminf(p.strength_log2 * ex * ex, p.cap_log2);
 }
 
-// How a thread treats its key block in the current tile.
+// How a row treats its key block in the current tile:
+//   mode 0  skip (the row's query block does not attend the block)
+//   mode 1  attended, no penalty
+//   mode 2  attended, penalty pen_a on keys [0, split) and pen_b on [split, 64)
+//           (log2 units; a block whose guide keys share one time, or two
+//           contiguous runs of guide / other keys)
+//   mode 3  attended, per-key penalty from the keys' guide times
 struct BlockMode {
-  int mode;     // 0 skip (not attended by this row), 1 plain, 2 constant penalty, 3 per-key penalty
-  int nv;       // valid keys of the block
-  int key0;     // first key (sequence row) of the block
-  float cpen;   // constant penalty (mode 2), log2 units
+  int mode, nv, key0, split;  // nv: valid keys; key0: first key (sequence row)
+  float pen_a, pen_b;
 };
 
 // Probabilities of 16 keys [c0, c0 + 16) of the thread's block, given the row
-// max m (log2 units), as 8 bf16 pairs; returns their fp32 sum.
-__device__ __forceinline__ float probs16(const float* s, const BlockMode& bm, int c0, float m, float scale,
-                                         float tq, const AttnParams& p, uint32_t* pk) {
+// max m (log2 units), as 8 bf16 pairs; they return their fp32 sum.
+//
+// Common case (every lane of the warp): modes 0 to 2 with all 16 keys valid.
+// The offset is -(m + constant penalty), or -inf for a block the row does not
+// attend (2^-inf = 0), so the three modes share one branch-free path; pairs are
+// scaled and offset by one f32x2 FMA and exponentiated on MUFU.
+__device__ __forceinline__ float probs16_fast(const float* s, float off, float scale, uint32_t* pk) {
+  const uint64_t scale2 = f2_pack(scale, scale), off2 = f2_pack(off, off);
+  uint64_t acc2[2] = {f2_pack(0.0f, 0.0f), f2_pack(0.0f, 0.0f)};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float a, b;
+    f2_unpack(f2_fma(f2_pack(s[2 * i], s[2 * i + 1]), scale2, off2), a, b);
+    a = ex2(a);
+    b = ex2(b);
+    acc2[i & 1] = f2_add(acc2[i & 1], f2_pack(a, b));
+    pk[i] = pack_bf16(a, b);
+  }
+  float a0, a1, b0, b1;
+  f2_unpack(acc2[0], a0, a1);
+  f2_unpack(acc2[1], b0, b1);
+  return (a0 + a1) + (b0 + b1);
+}
+
+// General case (rare: a block with per-key penalties -- guide keys of several
+// times, or guide and other keys mixed -- or the partial last block): each of
+// the 16 keys with its own validity and penalty.  A key's guide time comes from
+// gtime (NaN for a key that is not a guide key: the penalty formula then gives
+// max(NaN - window, 0) = 0), read as four broadcast 16-byte loads.
+__device__ __forceinline__ float probs16_general(const float* s, const BlockMode& bm, int c0, float m, float scale,
+                                                 float tq, const AttnParams& p, uint32_t* pk) {
   float lt = 0.0f;
-  if (bm.mode == 0) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) pk[i] = 0u;
-  } else if (bm.mode == 3) {
+  for (int q = 0; q < 4; ++q) {  // four keys at a time keeps few values live
+    float pen[4];
+    if (bm.mode == 3) {
+      const float4 t = __ldg(reinterpret_cast<const float4*>(p.gtime + bm.key0 + c0) + q);
+      pen[0] = block_penalty_log2(tq, t.x, p);
+      pen[1] = block_penalty_log2(tq, t.y, p);
+      pen[2] = block_penalty_log2(tq, t.z, p);
+      pen[3] = block_penalty_log2(tq, t.w, p);
+    } else {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float pp[2];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int col = c0 + 2 * i + e;
-        float pen_k = 0.0f;
-        if (col < bm.nv && p.seg[bm.key0 + col] == kSegGuide)
-          pen_k = block_penalty_log2(tq, p.times[bm.key0 + col], p);
-        pp[e] = col < bm.nv ? ex2(fmaf(s[2 * i + e], scale, -(m + pen_k))) : 0.0f;
-      }
-      lt += pp[0] + pp[1];
-      pk[i] = pack_bf16(pp[0], pp[1]);
+      for (int e = 0; e < 4; ++e) pen[e] = c0 + 4 * q + e < bm.split ? bm.pen_a : bm.pen_b;
     }
-  } else if (bm.nv >= c0 + 16) {
-    // pairs in packed fp32: scale and offset by one f32x2 FMA; one pair in
-    // four takes 2^x on the FMA pipe, the rest on MUFU
-    const float off = -(m + bm.cpen);
-    const uint64_t scale2 = f2_pack(scale, scale), off2 = f2_pack(off, off);
-    uint64_t acc2[2] = {f2_pack(0.0f, 0.0f), f2_pack(0.0f, 0.0f)};
+    float pp[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint64_t x2 = f2_fma(f2_pack(s[2 * i], s[2 * i + 1]), scale2, off2);
-      uint64_t p2;
-      if ((i & 3) == 3) {
-        p2 = ex2_poly2(x2);
-      } else {
-        float a, b;
-        f2_unpack(x2, a, b);
-        p2 = f2_pack(ex2(a), ex2(b));
-      }
-      acc2[i & 1] = f2_add(acc2[i & 1], p2);
-      float p0, p1;
-      f2_unpack(p2, p0, p1);
-      pk[i] = pack_bf16(p0, p1);
+    for (int e = 0; e < 4; ++e) {
+      const int col = c0 + 4 * q + e;
+      pp[e] = (bm.mode != 0 && col < bm.nv) ? ex2(fmaf(s[4 * q + e], scale, -(m + pen[e]))) : 0.0f;
     }
-    float a0, a1, b0, b1;
-    f2_unpack(acc2[0], a0, a1);
-    f2_unpack(acc2[1], b0, b1);
-    lt = (a0 + a1) + (b0 + b1);
-  } else {
-    const float off = -(m + bm.cpen);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int col = c0 + 2 * i;
-      const float p0 = col < bm.nv ? ex2(fmaf(s[2 * i], scale, off)) : 0.0f;
-      const float p1 = col + 1 < bm.nv ? ex2(fmaf(s[2 * i + 1], scale, off)) : 0.0f;
-      lt += p0 + p1;
-      pk[i] = pack_bf16(p0, p1);
-    }
+    lt += (pp[0] + pp[1]) + (pp[2] + pp[3]);
+    pk[2 * q] = pack_bf16(pp[0], pp[1]);
+    pk[2 * q + 1] = pack_bf16(pp[2], pp[3]);
   }
   return lt;
+}
+
+// Offset of a 16-key group on the fast path: -inf for a block the row does
+// not attend, else -(m + the group's penalty) (a fast block's penalty runs
+// split on a group boundary).
+__device__ __forceinline__ float fast_offset(const BlockMode& bm, int c0, float m) {
+  return bm.mode == 0 ? -INFINITY : -(m + (c0 < bm.split ? bm.pen_a : bm.pen_b));
+}
+
+// Maximum over N keys of a fully valid block (-inf if the row skips it).
+template <int N>
+__device__ __forceinline__ float full_max(const float* s, const BlockMode& bm) {
+  float mp[4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a) mp[a] = fmaxf(s[a], s[a + 4]);
+#pragma unroll
+  for (int i = 8; i < N; i += 8)
+#pragma unroll
+    for (int a = 0; a < 4; ++a) mp[a] = max3f(mp[a], s[i + a], s[i + 4 + a]);
+  return bm.mode == 0 ? -INFINITY : fmaxf(max3f(mp[0], mp[1], mp[2]), mp[3]);
 }
 
 // Maximum over the valid keys [c0, c0 + N) of the thread's block (-inf if none).
@@ -256,6 +277,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   int* n_entries_slot = reinterpret_cast<int*>(smem + L::kMisc + 8);
+  int* n_fast_slot = reinterpret_cast<int*>(smem + L::kMisc + 12);
   const int nwords = (p.n_blocks + 31) >> 5;
   uint32_t* bm_a = reinterpret_cast<uint32_t*>(smem + L::kBitmaps);
   uint32_t* bm_b = bm_a + nwords;
@@ -334,28 +356,40 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
   __syncthreads();
   if (warp == 0) {
-    // lane l owns words [l*per, (l+1)*per)
+    // Entries in ascending block order, except that the blocks needing
+    // per-key treatment (p.slow_blocks) go after all the others; the online
+    // softmax may visit key blocks in any order.  Lane l owns words
+    // [l*per, (l+1)*per); fast and slow counts share one scan (16 bits each).
     const int per = (nwords + 31) / 32;
     const int w0 = lane * per, w1 = min(nwords, (lane + 1) * per);
     int cnt = 0;
-    for (int w = w0; w < w1; ++w) cnt += __popc(bm_a[w] | bm_b[w]);
+    for (int w = w0; w < w1; ++w) {
+      const uint32_t u = bm_a[w] | bm_b[w], slow = p.slow_blocks[w];
+      cnt += __popc(u & ~slow) | (__popc(u & slow) << 16);
+    }
     int incl = cnt;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int v = __shfl_up_sync(kFull, incl, o);
       if (lane >= o) incl += v;
     }
-    int pos = incl - cnt;
+    const int n_fast = __shfl_sync(kFull, incl, 31) & 0xFFFF;
+    int pos_f = (incl - cnt) & 0xFFFF, pos_s = n_fast + ((incl - cnt) >> 16);
     for (int w = w0; w < w1; ++w) {
-      const uint32_t a = bm_a[w], b = bm_b[w];
+      const uint32_t a = bm_a[w], b = bm_b[w], slow = p.slow_blocks[w];
       uint32_t u = a | b;
       while (u) {
         const int bit = __ffs(u) - 1;
         u &= u - 1;
-        list[pos++] = (uint16_t)((w * 32 + bit) | (((a >> bit) & 1u) << 14) | (((b >> bit) & 1u) << 15));
+        const uint16_t e = (uint16_t)((w * 32 + bit) | (((a >> bit) & 1u) << 14) | (((b >> bit) & 1u) << 15));
+        if ((slow >> bit) & 1u) list[pos_s++] = e;
+        else list[pos_f++] = e;
       }
     }
-    if (lane == 31) *n_entries_slot = incl;
+    if (lane == 31) {
+      *n_entries_slot = (incl & 0xFFFF) + (incl >> 16);
+      *n_fast_slot = incl & 0xFFFF;
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -363,6 +397,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t tmem_base = *tmem_base_slot;
   const int n_entries = *n_entries_slot;
   const int n_tiles = (n_entries + 1) >> 1;
+  const int n_fast_tiles = *n_fast_slot >> 1;  // tiles whose two blocks are both fast
 
   if (warp < 2) {
     if (warp == 0 && lane == 0) {
@@ -530,28 +565,34 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     };
 
-    for (int j = 0; ok && j < n_tiles; ++j) {
+    // One tile; kGeneral selects the per-key path (validity, per-key penalty)
+    // that the few slow key blocks need -- kept out of the loop over the
+    // others so that it does not weigh on their register allocation.
+    auto tile = [&](int j, auto general) -> bool {
+      constexpr bool kGeneral = decltype(general)::value;
       const uint32_t ph = (uint32_t)j & 1u;
       // this thread's key block and its descriptor, fetched before the wait
       const int idx = 2 * j + part;
       const uint32_t ent = idx < n_entries ? (uint32_t)list[idx] : 0u;
       const bool attended = idx < n_entries && ((ent >> my_bit) & 1u);
-      const uint2 kd = attended ? __ldg(p.kv_desc + (ent & 0x3FFFu)) : make_uint2(0u, 0u);
-      BlockMode bm{0, 0, (int)(ent & 0x3FFFu) * 64, 0.0f};
+      const uint4 kd = attended ? __ldg(p.kv_desc + (ent & 0x3FFFu)) : make_uint4(0u, 0u, 0u, 0u);
+      BlockMode bm{0, 0, (int)(ent & 0x3FFFu) * 64, 64, 0.0f, 0.0f};
       if (attended) {
         bm.nv = (int)(kd.x & 0xFFu);
         const int kind = (int)((kd.x >> 8) & 3u);
         bm.mode = 1;
         if (pen_row && kind == 1) {
-          bm.cpen = block_penalty_log2(tq, __uint_as_float(kd.y), p);
+          // a non-guide run has time NaN: its penalty evaluates to 0
+          bm.split = (int)((kd.x >> 16) & 0xFFu);
+          bm.pen_a = block_penalty_log2(tq, __uint_as_float(kd.y), p);
+          bm.pen_b = bm.split < bm.nv ? block_penalty_log2(tq, __uint_as_float(kd.z), p) : bm.pen_a;
           bm.mode = 2;
         } else if (pen_row && kind == 2) {
           bm.mode = 3;
         }
       }
       if (!__all_sync(kFull, wait_bar(bars.s_full, ph, p, abort_flag))) {
-        ok = false;
-        break;
+        return false;
       }
       tc_fence_after();
 
@@ -569,9 +610,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int i = 0; i < 16; ++i) sv[32 + i] = __uint_as_float(t16[i]);
       }
       float mx;
-      if (!exchange_max(part_max<kPhase0Keys>(sv, bm, 0), 0, mx)) {
-        ok = false;
-        break;
+      if (!exchange_max(kGeneral ? part_max<kPhase0Keys>(sv, bm, 0) : full_max<kPhase0Keys>(sv, bm), 0, mx)) {
+        return false;
       }
       // Conditional rescale: the running max only moves when it grows by more
       // than 2^8; below that the stale max keeps every probability <= 256.
@@ -583,7 +623,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
       for (int g = 0; g < kPhase0Keys / 16; ++g) {
         uint32_t pk[8];
-        lt += probs16(sv + 16 * g, bm, 16 * g, m, scale, tq, p, pk);
+        lt += kGeneral ? probs16_general(sv + 16 * g, bm, 16 * g, m, scale, tq, p, pk)
+                       : probs16_fast(sv + 16 * g, fast_offset(bm, 16 * g, m), scale, pk);
         __syncwarp();
         tmem_st8(t_s + 8 * g, pk);  // P of keys 16g..16g+15 over score columns 8g..8g+7
       }
@@ -601,8 +642,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       // O is stable once PV(j-1, phase 1) has completed (waited on every tile)
       if (j > 0) {
         if (!__all_sync(kFull, wait_bar(bars.o_done, ph ^ 1u, p, abort_flag))) {
-          ok = false;
-          break;
+          return false;
         }
         tc_fence_after();
       }
@@ -618,26 +658,25 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (lane == 0) mbar_arrive(bars.p_full);  // one arrival per softmax warp
 
       // ---------------- phase 1: keys 48..63, P to shared memory
-      if (!exchange_max(part_max<16>(sv1, bm, kPhase0Keys), 1, mx)) {
-        ok = false;
-        break;
+      if (!exchange_max(kGeneral ? part_max<16>(sv1, bm, kPhase0Keys) : full_max<16>(sv1, bm), 1, mx)) {
+        return false;
       }
       grow = mx > m + kRescaleThreshold;
       o_rescale = grow && m > -INFINITY;
       m_old = m;
       if (grow) m = mx;
       {
-        uint32_t pk[8];
-        lt = probs16(sv1, bm, kPhase0Keys, m, scale, tq, p, pk);
         // PV(j-1, phase 1) read the previous contents: complete (o_done above)
+        uint32_t pk[8];
+        lt = kGeneral ? probs16_general(sv1, bm, kPhase0Keys, m, scale, tq, p, pk)
+                      : probs16_fast(sv1, fast_offset(bm, kPhase0Keys, m), scale, pk);
         *reinterpret_cast<uint4*>(ph1_row + (0u ^ ph1_swz)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         *reinterpret_cast<uint4*>(ph1_row + (16u ^ ph1_swz)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
       }
       fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor core
       alpha = 1.0f;
       if (!__all_sync(kFull, wait_bar(bars.o_half0, ph, p, abort_flag))) {
-        ok = false;
-        break;
+        return false;
       }
       tc_fence_after();
       if (__any_sync(kFull, o_rescale)) {
@@ -649,7 +688,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.p_full + 1);
-    }
+      return true;
+    };
+    int j = 0;
+    for (; ok && j < n_fast_tiles; ++j) ok = tile(j, std::false_type{});
+    for (; ok && j < n_tiles; ++j) ok = tile(j, std::true_type{});
     // ---------------------------------------------------------- epilogue
     bool fin = __all_sync(kFull, ok) && n_tiles > 0;
     // total row sum: slot 0 is free here (its last reader passed the barrier

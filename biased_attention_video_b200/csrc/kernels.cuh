@@ -21,7 +21,9 @@ struct AttnParams {
   const int32_t* kv_sel;       // [H][nV][k] or null (dense)
   const uint8_t* seg;          // [S]
   const float* times;          // [S]
-  const uint2* kv_desc;        // [n_blocks]: x = valid rows | kind << 8, y = time bits (kind 1)
+  const uint4* kv_desc;        // [n_blocks]: see launch_kv_desc
+  const float* gtime;          // [n_blocks * 64]: guide key's time, NaN for other keys (read for kind 2)
+  const uint32_t* slow_blocks; // [ceil(n_blocks / 32)] bitmap: blocks needing per-key treatment
   uint16_t* o;                 // bf16 [H][S][d]
   float* lse;                  // [H][S] or null
   int* status;                 // device status word
@@ -36,9 +38,19 @@ int attn_smem_bytes(int d, int n_blocks);
 cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                         const AttnParams& p, int n_ctas, cudaStream_t stream);
 
-// kv_desc[b] for every key block (valid rows, guide-key kind, uniform time)
-cudaError_t launch_kv_desc(const uint8_t* seg, const float* times, int S, int n_blocks, uint2* kv_desc,
-                           cudaStream_t stream);
+// kv_desc[b] for every key block b, over its valid rows (n of them):
+//   x = n | kind << 8 | split << 16, y / z = time bits of runs a / b
+//   kind 0: no guide row;
+//   kind 1: rows [0, split) and [split, n) each all guide rows of one time
+//           (y, z) or all other rows (time NaN); split = n for a single run;
+//   kind 2: anything else (per-row times needed).
+// And, when times is not null, gtime[r] for every row r < 64 n_blocks: the
+// row's time if it is a guide row below S, NaN otherwise.
+// slow[b / 32] bit b % 32: block b needs per-key treatment in the attention
+// kernel (fewer than 64 valid rows, kind 2, or a kind-1 split inside a
+// 16-key group), for every block b < 32 ceil(n_blocks / 32).
+cudaError_t launch_kv_desc(const uint8_t* seg, const float* times, int S, int n_blocks, uint4* kv_desc,
+                           float* gtime, uint32_t* slow, cudaStream_t stream);
 
 // mean-pool blocks [first_block, first_block + n_out) of up to two bf16 [H][S][d] tensors
 cudaError_t launch_pool(const uint16_t* x0, float* out0, const uint16_t* x1, float* out1, int H, int S,
@@ -63,6 +75,5 @@ cudaError_t launch_route_pipeline(const uint16_t* q, const uint16_t* k, int32_t*
                                   cudaStream_t stream);
 
 cudaError_t launch_selftest_timeout(int* status, uint32_t polls, cudaStream_t stream);
-cudaError_t launch_selftest_exp2(const float* x, float* y, int n_pairs, cudaStream_t stream);
 
 }  // namespace h3

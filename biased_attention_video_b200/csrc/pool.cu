@@ -78,24 +78,44 @@ __global__ void __launch_bounds__(256) pool_kernel(const uint16_t* __restrict__ 
 // row is a guide row and all share one time (stored in .y), 2: anything else
 // holding guide rows (penalty evaluated per key).
 __global__ void kv_desc_kernel(const uint8_t* __restrict__ seg, const float* __restrict__ times, int S,
-                               int n_blocks, uint2* __restrict__ desc) {
-  const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b >= n_blocks) return;
-  const int lo = b * kBlock;
-  const int n = min(kBlock, S - lo);
-  int guides = 0;
-  bool same_time = true;
-  float t0 = 0.0f;
-  for (int r = 0; r < n; ++r) {
-    if (seg[lo + r] == kSegGuide) {
-      const float t = times != nullptr ? times[lo + r] : 0.0f;
-      if (guides == 0) t0 = t;
-      else if (t != t0) same_time = false;
-      ++guides;
+                               int n_blocks, uint4* __restrict__ desc, float* __restrict__ gtime,
+                               uint32_t* __restrict__ slow_bits) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;  // 32 consecutive blocks per warp
+  bool slow = false;
+  if (b < n_blocks) {
+    const int lo = b * kBlock;
+    const int n = min(kBlock, S - lo);
+    const float nan = __int_as_float(0x7FC00000);
+    // each row's key time: its time if it is a guide row, NaN otherwise; the
+    // block splits into at most two runs of equal key time (NaN == NaN here)
+    bool any_guide = false, two_runs = true;
+    int split = n;
+    uint32_t ta = 0u, tb = 0u;
+    for (int r = 0; r < kBlock; ++r) {
+      const bool guide = r < n && seg[lo + r] == kSegGuide;
+      const float t = guide ? (times != nullptr ? times[lo + r] : 0.0f) : nan;
+      if (gtime != nullptr && times != nullptr) gtime[lo + r] = t;
+      if (r >= n) continue;
+      any_guide |= guide;
+      const uint32_t tbits = __float_as_uint(t);
+      if (r == 0) {
+        ta = tb = tbits;
+      } else if (split == n) {
+        if (tbits != ta) {
+          split = r;
+          tb = tbits;
+        }
+      } else if (tbits != tb) {
+        two_runs = false;
+      }
     }
+    const uint32_t kind = !any_guide ? 0u : (two_runs ? 1u : 2u);
+    desc[b] = make_uint4((uint32_t)n | (kind << 8) | ((uint32_t)split << 16), ta, tb, 0u);
+    // (penalty off -- times null -- leaves only the validity test)
+    slow = n < kBlock || (times != nullptr && (kind == 2u || (kind == 1u && split < n && (split & 15) != 0)));
   }
-  uint32_t kind = guides == 0 ? 0u : ((guides == n && same_time) ? 1u : 2u);
-  desc[b] = make_uint2((uint32_t)n | (kind << 8), __float_as_uint(t0));
+  const uint32_t word = __ballot_sync(0xFFFFFFFFu, slow);
+  if ((threadIdx.x & 31) == 0 && b < ((n_blocks + 31) & ~31)) slow_bits[b >> 5] = word;
 }
 
 __global__ void selftest_timeout_kernel(int* status, uint32_t polls) {
@@ -109,21 +129,8 @@ __global__ void selftest_timeout_kernel(int* status, uint32_t polls) {
   }
 }
 
-__global__ void selftest_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, int n_pairs) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n_pairs) return;
-  float a, b;
-  f2_unpack(ex2_poly2(f2_pack(x[2 * i], x[2 * i + 1])), a, b);
-  y[2 * i] = a;
-  y[2 * i + 1] = b;
-}
-
 }  // namespace
 
-cudaError_t launch_selftest_exp2(const float* x, float* y, int n_pairs, cudaStream_t stream) {
-  if (n_pairs > 0) selftest_exp2_kernel<<<(n_pairs + 255) / 256, 256, 0, stream>>>(x, y, n_pairs);
-  return cudaGetLastError();
-}
 
 cudaError_t launch_pool(const uint16_t* x0, float* out0, const uint16_t* x1, float* out1, int H, int S, int d,
                         int first_block, int n_out, cudaStream_t stream) {
@@ -137,9 +144,9 @@ cudaError_t launch_pool(const uint16_t* x0, float* out0, const uint16_t* x1, flo
   return cudaGetLastError();
 }
 
-cudaError_t launch_kv_desc(const uint8_t* seg, const float* times, int S, int n_blocks, uint2* kv_desc,
-                           cudaStream_t stream) {
-  kv_desc_kernel<<<(n_blocks + 127) / 128, 128, 0, stream>>>(seg, times, S, n_blocks, kv_desc);
+cudaError_t launch_kv_desc(const uint8_t* seg, const float* times, int S, int n_blocks, uint4* kv_desc,
+                           float* gtime, uint32_t* slow, cudaStream_t stream) {
+  kv_desc_kernel<<<(n_blocks + 127) / 128, 128, 0, stream>>>(seg, times, S, n_blocks, kv_desc, gtime, slow);
   return cudaGetLastError();
 }
 

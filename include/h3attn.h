@@ -115,9 +115,11 @@ H3ATTN_API int h3attn_plan_init(h3attn_plan* plan, int H, int S, int d, int bloc
                      const uint8_t* seg_host);
 
 /* Bytes of device workspace a plan needs for h3attn_route and h3attn_forward
- * (status word, per-block key descriptors, and the routing scratch: two-part
- * bf16 pooled Q and K of the video blocks and the fp32 pooled-score matrix,
- * about 0.9 GB at S = 116,883, H = 56, d = 128).
+ * (status word; the attention scratch: per-block key descriptors, per-key
+ * guide times and a bitmap of the key blocks that need per-key handling,
+ * about 0.5 MB at S = 116,883; and the routing scratch: two-part bf16 pooled
+ * Q and K of the video blocks and the fp32 pooled-score matrix, about 0.9 GB
+ * at S = 116,883, H = 56, d = 128).
  * The caller allocates it once, zero-filled (the first 256 bytes hold the
  * status word that h3attn_check reads and clears). */
 H3ATTN_API size_t h3attn_workspace_bytes(const h3attn_plan* plan);
@@ -177,7 +179,8 @@ H3ATTN_API int h3attn_forward(const h3attn_plan* plan, const uint16_t* q, const 
 
 /* Dense biased attention (every query attends every key; the penalty on
  * output -> guide pairs): h3attn_forward with a dense plan and kv_sel NULL.
- * Needs h3attn_dense_workspace_bytes(S) bytes of zero-filled workspace. */
+ * Needs h3attn_dense_workspace_bytes(S) bytes of zero-filled workspace (the
+ * status word and the attention scratch). */
 H3ATTN_API size_t h3attn_dense_workspace_bytes(int S);
 H3ATTN_API int h3attn_dense_biased(int H, int S, int d, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                         const uint8_t* seg, const float* times, const h3attn_penalty* pen, uint16_t* o,
@@ -192,12 +195,6 @@ H3ATTN_API int h3attn_check(void* ws, void* stream);
  * an mbarrier nothing arrives at, with a limit of `polls` polls, and records
  * H3ATTN_ETIMEOUT in the status word when it gives up.  No other work. */
 H3ATTN_API int h3attn_selftest_timeout(void* ws, uint32_t polls, void* stream);
-
-/* Self-test of the softmax's FMA-pipe exponential: y[i] = 2^x[i] computed
- * the way the attention kernel computes one pair in four of its
- * probabilities (inputs below -125 are clamped to -125).  x, y: float32 [n]
- * device, n even, 8-byte aligned. */
-H3ATTN_API int h3attn_selftest_exp2(const float* x, float* y, int n, void* stream);
 
 /* Static description of a status code (never NULL). */
 H3ATTN_API const char* h3attn_strerror(int status);
