@@ -6,8 +6,8 @@ penalty (workload "full combined").
 Prints one JSON line.  value = effective attention TFLOP/s over all ranks
 (4*d FLOPs per attended (query, key, head) triple, valid pairs only) with the
 inputs resident in HBM; e2e = the same metric through the C ABI with host
-buffers (host->device copy of Q, K, V, seg, times and device->host copy of O
-inside the timed region).
+buffers (h3attn_attend_host: host->device copy of Q, K, V, seg, times and
+device->host copy of O inside the timed region, pipelined per chunk of heads).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Multi-GPU: torchrun, one process per GPU; every rank runs its own independent
@@ -331,15 +331,13 @@ def run_ours(args, rank, world, local_rank):
     d2h = n * 2
     qh_v, kh_v, vh_v = host["q"], host["k"], host["v"]
 
+    # the public host-buffer call: head chunks pipelined over three streams
+    copy_in, copy_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
     def e2e_step():
-        qd.view(torch.int16).view(-1).copy_(qh_v, non_blocking=True)
-        kd.view(torch.int16).view(-1).copy_(kh_v, non_blocking=True)
-        vd.view(torch.int16).view(-1).copy_(vh_v, non_blocking=True)
-        seg_d.copy_(seg_h, non_blocking=True)
-        times_d.copy_(times_h, non_blocking=True)
-        h3.route(p, qd, kd, ws, kv_sel=sel)
-        h3.forward(p, qd, kd, vd, seg_d, times_d, pen=pen, kv_sel=sel, ws=ws, out=o)
-        o_h.copy_(o.view(torch.int16).view(-1), non_blocking=True)
+        h3.attend_host(p, qh_v, kh_v, vh_v, seg_h, times_h, o_h, q=qd, k=kd, v=vd, seg=seg_d, times=times_d, o=o,
+                       ws=ws, kv_sel=sel, pen=pen, chunk_heads=min(args.chunk_heads, H), stream=stream,
+                       copy_in_stream=copy_in, copy_out_stream=copy_out)
 
     e2e_ms = float("nan")
     if not args.no_e2e:
@@ -417,6 +415,7 @@ def main():
     ap.add_argument("--heads", type=int, default=None,
                     help="run the same packing with fewer heads (profiling captures only; the default is 56)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--chunk-heads", type=int, default=2, help="heads per pipelined chunk of the host-buffer call")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -26,7 +26,7 @@ SEG_TEXT, SEG_IMAGE_REF, SEG_AUDIO, SEG_GUIDE, SEG_OUTPUT = 0, 1, 2, 3, 4
 EXPORTS = ("h3attn_plan_init", "h3attn_workspace_bytes", "h3attn_pool", "h3attn_route", "h3attn_route_static",
            "h3attn_forward",
            "h3attn_dense_workspace_bytes", "h3attn_dense_biased", "h3attn_check", "h3attn_selftest_timeout",
-           "h3attn_strerror")
+           "h3attn_attend_host", "h3attn_strerror")
 
 
 class H3Error(RuntimeError):
@@ -85,6 +85,9 @@ def lib():
         L.h3attn_dense_biased.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, _P,
                                           ctypes.POINTER(Penalty), _P, _P, _P, ctypes.c_size_t, _P]
         L.h3attn_dense_biased.restype = ctypes.c_int
+        L.h3attn_attend_host.argtypes = [PP, _P, _P, _P, _P, _P, ctypes.POINTER(Penalty), _P, _P, _P, _P, _P, _P,
+                                         _P, _P, _P, _P, _P, ctypes.c_size_t, ctypes.c_int, _P, _P, _P]
+        L.h3attn_attend_host.restype = ctypes.c_int
         L.h3attn_check.argtypes = [_P, _P]
         L.h3attn_check.restype = ctypes.c_int
         L.h3attn_selftest_timeout.argtypes = [_P, ctypes.c_uint32, _P]
@@ -208,6 +211,23 @@ def dense_biased(q, k, v, seg, times, pen=DEFAULT_PENALTY, ws=None, out=None, ls
                                      _dptr(times), ctypes.byref(pn) if pn is not None else None, o.data_ptr(),
                                      _dptr(lse_t), ws.data_ptr(), ws.numel(), _stream(stream)), "dense_biased")
     return o, lse_t
+
+
+def attend_host(p: Plan, q_host, k_host, v_host, seg_host, times_host, o_host, *, q, k, v, seg, times, o, ws,
+                kv_sel=None, pen=DEFAULT_PENALTY, lse_host=None, lse=None, chunk_heads: int = 4, stream=None,
+                copy_in_stream=None, copy_out_stream=None) -> None:
+    """The whole call from (page-locked) host tensors, copies overlapped with the kernels per chunk of heads.
+
+    Host tensors: q_host/k_host/v_host/o_host bf16 or int16 [H, S, d]; seg_host uint8 [S]; times_host float32 [S];
+    device buffers q/k/v/o/seg/times (and kv_sel, lse) of the same shapes.  Streams are torch.cuda.Stream
+    objects (None = the current stream)."""
+    pn = _pen(pen)
+    _raise(lib().h3attn_attend_host(
+        ctypes.byref(p), q_host.data_ptr(), k_host.data_ptr(), v_host.data_ptr(), seg_host.data_ptr(),
+        _dptr(times_host), ctypes.byref(pn) if pn is not None else None, o_host.data_ptr(), _dptr(lse_host),
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), seg.data_ptr(), _dptr(times), _dptr(kv_sel), o.data_ptr(),
+        _dptr(lse), ws.data_ptr(), ws.numel(), chunk_heads, _stream(stream), _stream(copy_in_stream),
+        _stream(copy_out_stream)), "attend_host")
 
 
 def check(ws: torch.Tensor, stream=None) -> int:

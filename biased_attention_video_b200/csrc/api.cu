@@ -1,9 +1,11 @@
+#include <algorithm>
 // C ABI of libh3attn: argument validation, block plan, workspace layout,
 // TMA descriptors and kernel launches.  See include/h3attn.h for the contract.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <new>
 #include <cstdint>
 #include <cstring>
 
@@ -237,6 +239,89 @@ int h3attn_forward(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k
   if (kv_sel != nullptr && (reinterpret_cast<uintptr_t>(kv_sel) & 3u)) return H3ATTN_EALIGN;
   return forward_impl(plan, q, k, v, seg, times, pen, kv_sel, o, lse, ws, ws_bytes, need,
                       static_cast<cudaStream_t>(stream));
+}
+
+int h3attn_attend_host(const h3attn_plan* plan, const uint16_t* q_host, const uint16_t* k_host,
+                       const uint16_t* v_host, const uint8_t* seg_host, const float* times_host,
+                       const h3attn_penalty* pen, uint16_t* o_host, float* lse_host, uint16_t* q, uint16_t* k,
+                       uint16_t* v, uint8_t* seg, float* times, int32_t* kv_sel, uint16_t* o, float* lse, void* ws,
+                       size_t ws_bytes, int chunk_heads, void* stream, void* copy_in_stream,
+                       void* copy_out_stream) {
+  if (!plan_ok(plan)) return H3ATTN_EINVAL;
+  if (!q_host || !k_host || !v_host || !seg_host || !o_host || !q || !k || !v || !seg || !o) return H3ATTN_EINVAL;
+  const bool routed = plan->n_video_blocks > 0 && plan->k < plan->n_video_blocks;
+  if (routed && kv_sel == nullptr) return H3ATTN_EINVAL;
+  if ((lse_host == nullptr) != (lse == nullptr)) return H3ATTN_EINVAL;
+  if (pen != nullptr && (times_host == nullptr || times == nullptr)) return H3ATTN_EINVAL;
+  if (chunk_heads < 1 || chunk_heads > plan->H) return H3ATTN_EINVAL;
+  if (ws == nullptr || ws_bytes < h3attn_workspace_bytes(plan)) return H3ATTN_EWORKSPACE;
+  const cudaStream_t sc = static_cast<cudaStream_t>(stream);
+  const cudaStream_t si = static_cast<cudaStream_t>(copy_in_stream);
+  const cudaStream_t so = static_cast<cudaStream_t>(copy_out_stream);
+  const size_t per_head = (size_t)plan->S * plan->d;  // elements of one head of Q/K/V/O
+  const size_t sel_per_head = (size_t)plan->n_video_blocks * plan->k;
+  const int n_chunks = (plan->H + chunk_heads - 1) / chunk_heads;
+  // two events per chunk (inputs landed, outputs ready), one for the end and
+  // one for the start
+  const int n_events = 2 * n_chunks + 2;
+  cudaEvent_t* evs = new (std::nothrow) cudaEvent_t[n_events];
+  if (evs == nullptr) return H3ATTN_ECUDA;
+  int n_ev = 0, rc = H3ATTN_OK;
+  for (; n_ev < n_events; ++n_ev)
+    if (cudaEventCreateWithFlags(&evs[n_ev], cudaEventDisableTiming) != cudaSuccess) {
+      rc = H3ATTN_ECUDA;
+      break;
+    }
+  auto copy = [&](void* dst, const void* src, size_t bytes, cudaMemcpyKind kind, cudaStream_t st) {
+    if (rc == H3ATTN_OK && cudaMemcpyAsync(dst, src, bytes, kind, st) != cudaSuccess) rc = H3ATTN_ECUDA;
+  };
+  auto record = [&](cudaEvent_t e, cudaStream_t st) {
+    if (rc == H3ATTN_OK && cudaEventRecord(e, st) != cudaSuccess) rc = H3ATTN_ECUDA;
+  };
+  auto wait = [&](cudaStream_t st, cudaEvent_t e) {
+    if (rc == H3ATTN_OK && cudaStreamWaitEvent(st, e, 0) != cudaSuccess) rc = H3ATTN_ECUDA;
+  };
+  // the copies start once `stream` has reached this call: work queued there
+  // before (an earlier call still reading or writing these buffers) is done
+  record(evs[2 * n_chunks + 1], sc);
+  wait(si, evs[2 * n_chunks + 1]);
+  wait(so, evs[2 * n_chunks + 1]);
+  // the per-sequence inputs go first, with the first chunk
+  copy(seg, seg_host, (size_t)plan->S, cudaMemcpyHostToDevice, si);
+  if (times_host != nullptr && times != nullptr)
+    copy(times, times_host, (size_t)plan->S * sizeof(float), cudaMemcpyHostToDevice, si);
+  for (int c = 0; c < n_chunks && rc == H3ATTN_OK; ++c) {
+    const int h0 = c * chunk_heads, hc = std::min(chunk_heads, plan->H - h0);
+    const size_t off = (size_t)h0 * per_head, bytes = (size_t)hc * per_head * sizeof(uint16_t);
+    copy(q + off, q_host + off, bytes, cudaMemcpyHostToDevice, si);
+    copy(k + off, k_host + off, bytes, cudaMemcpyHostToDevice, si);
+    copy(v + off, v_host + off, bytes, cudaMemcpyHostToDevice, si);
+    record(evs[2 * c], si);
+    wait(sc, evs[2 * c]);
+    if (rc != H3ATTN_OK) break;
+    h3attn_plan cp = *plan;  // the same sequence, hc heads
+    cp.H = hc;
+    int32_t* sel = routed ? kv_sel + (size_t)h0 * sel_per_head : nullptr;
+    if (routed) {
+      rc = h3attn_route(&cp, q + off, k + off, sel, ws, ws_bytes, stream);
+      if (rc != H3ATTN_OK) break;
+    }
+    rc = h3attn_forward(&cp, q + off, k + off, v + off, seg, times, pen, sel, o + off,
+                        lse != nullptr ? lse + (size_t)h0 * plan->S : nullptr, ws, ws_bytes, stream);
+    if (rc != H3ATTN_OK) break;
+    record(evs[2 * c + 1], sc);
+    wait(so, evs[2 * c + 1]);
+    copy(o_host + off, o + off, bytes, cudaMemcpyDeviceToHost, so);
+    if (lse != nullptr)
+      copy(lse_host + (size_t)h0 * plan->S, lse + (size_t)h0 * plan->S, (size_t)hc * plan->S * sizeof(float),
+           cudaMemcpyDeviceToHost, so);
+  }
+  // the caller's stream completes after the last copy back
+  record(evs[2 * n_chunks], so);
+  wait(sc, evs[2 * n_chunks]);
+  for (int i = 0; i < n_ev; ++i) cudaEventDestroy(evs[i]);  // released once their work is done
+  delete[] evs;
+  return rc;
 }
 
 size_t h3attn_dense_workspace_bytes(int S) {

@@ -177,6 +177,37 @@ H3ATTN_API int h3attn_forward(const h3attn_plan* plan, const uint16_t* q, const 
                    const int32_t* kv_sel, uint16_t* o, float* lse, void* ws, size_t ws_bytes,
                    void* stream);
 
+/* The whole call from host memory: routing (when the plan routes) and
+ * attention for every head, with the host<->device copies overlapped with the
+ * kernels.  Every step of the path is independent per head ("H3 SLA
+ * Attention", "How it works": routing per head; the attention is per head),
+ * so the heads go in chunks of chunk_heads: chunk c's Q/K/V copy in on
+ * copy_in_stream, its routing and attention run on `stream` once they have
+ * landed, and its O (and LSE) copy out on copy_out_stream, while chunk c+1 is
+ * already copying in.
+ *  q_host, k_host, v_host: bf16 [H][S][d]; o_host: bf16 [H][S][d];
+ *  seg_host: uint8 [S]; times_host: float32 [S] (may be NULL when pen is NULL);
+ *  lse_host: float32 [H][S] or NULL -- host memory, page-locked for the copies
+ *  to overlap (pageable memory works but serialises).
+ *  q, k, v, o: device buffers of the same shapes; seg, times: device [S];
+ *  kv_sel: device int32 [H][n_video_blocks][k] (may be NULL when the plan does
+ *  not route); lse: device float32 [H][S], NULL exactly when lse_host is.
+ *  ws: as for h3attn_route / h3attn_forward (h3attn_workspace_bytes(plan)).
+ *  Results: o_host / lse_host as h3attn_forward would give; they are complete
+ *  when `stream` reaches the point where this call returns (the call makes
+ *  `stream` wait for the last copy out).  The copies start only after the work
+ *  already queued on `stream`, so back-to-back calls on the same buffers do
+ *  not overlap one another.  Three distinct streams give the
+ *  overlap; the same stream three times gives the same results in sequence.
+ *  Errors as for h3attn_route / h3attn_forward, checked before each chunk's
+ *  launches; chunk_heads must lie in [1, H]. */
+H3ATTN_API int h3attn_attend_host(const h3attn_plan* plan, const uint16_t* q_host, const uint16_t* k_host,
+                                  const uint16_t* v_host, const uint8_t* seg_host, const float* times_host,
+                                  const h3attn_penalty* pen, uint16_t* o_host, float* lse_host, uint16_t* q,
+                                  uint16_t* k, uint16_t* v, uint8_t* seg, float* times, int32_t* kv_sel, uint16_t* o,
+                                  float* lse, void* ws, size_t ws_bytes, int chunk_heads, void* stream,
+                                  void* copy_in_stream, void* copy_out_stream);
+
 /* Dense biased attention (every query attends every key; the penalty on
  * output -> guide pairs): h3attn_forward with a dense plan and kv_sel NULL.
  * Needs h3attn_dense_workspace_bytes(S) bytes of zero-filled workspace (the

@@ -117,6 +117,14 @@ def test_host_validation_before_any_device_work():
     assert L.h3attn_pool(ctypes.byref(p), fake, 2, 9, fake, None) == h3.EINVAL
     assert L.h3attn_dense_biased(1, 256, 80, fake, fake, fake, fake, fake, None, fake, None, fake, 1 << 20,
                                  None) == h3.EUNSUPPORTED
+    # host-buffer pipeline: argument checks come before any copy or launch
+    args = [fake] * 17
+    assert L.h3attn_attend_host(ctypes.byref(p), *args[:5], None, *args[5:16], ws_need, 0, None, None,
+                                None) == h3.EINVAL  # chunk_heads 0
+    assert L.h3attn_attend_host(ctypes.byref(p), *args[:5], None, *args[5:16], ws_need, 2, None, None,
+                                None) == h3.EINVAL  # chunk_heads > H
+    assert L.h3attn_attend_host(ctypes.byref(p), *args[:5], None, *args[5:16], 16, 1, None, None,
+                                None) == h3.EWORKSPACE
     p.k = 0  # corrupt plan
     assert L.h3attn_workspace_bytes(ctypes.byref(p)) == 0
     for code in [0, -1, -2, -3, -4, -5, -6, -7, -99]:
