@@ -116,6 +116,26 @@ def max_over_ranks(values, world: int, device="cpu"):
     return [float(x) for x in t.cpu()]
 
 
+def head_range(H: int, world: int, rank: int):
+    """Heads [h0, h0 + nh) of rank `rank` when one call's H heads are split over `world` ranks: contiguous,
+    sizes differing by at most one, together covering every head once.  Every step of the path is
+    independent per head, so the shards need no collective."""
+    base, extra = divmod(H, world)
+    nh = base + (1 if rank < extra else 0)
+    h0 = rank * base + min(rank, extra)
+    return h0, nh
+
+
+def sum_over_ranks(values, world: int, device="cpu"):
+    """Element-wise sum over ranks (no-op for one rank)."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return [float(x) for x in t.cpu()]
+
+
 def whole_job_tflops(flops_per_call: float, calls_per_rank: int, world: int, ms: float) -> float:
     """Aggregate throughput of all ranks: every rank did calls_per_rank calls in at most ms."""
     return world * flops_per_call * calls_per_rank / (ms * 1e-3) / 1e12
@@ -255,9 +275,15 @@ def run_ours(args, rank, world, local_rank):
     if args.heads is not None:
         cfg = inputs.custom(args.heads, cfg.d, cfg.segments, cfg.seed, cluster_norm=cfg.cluster_norm,
                             penalty=cfg.penalty, sparsities=cfg.sparsities, name=f"{cfg.name} ({args.heads} heads)")
-    seed = rank_seed(cfg.seed, rank)
+    sharded = args.shard == "heads"
+    # weak scaling: every rank its own independent call (seed shifted by the rank); head sharding: one call
+    # (one seed), each rank its contiguous range of heads
+    seed = cfg.seed if sharded else rank_seed(cfg.seed, rank)
     seg, times, _ = cfg.layout()
-    H, S, d = cfg.H, cfg.S, cfg.d
+    if sharded and world > cfg.H:
+        raise SystemExit(f"--shard heads needs at most {cfg.H} ranks")
+    h0, H = head_range(cfg.H, world, rank) if sharded else (0, cfg.H)
+    S, d = cfg.S, cfg.d
     sparsity = cfg.sparsities[0]
     pen = cfg.penalty
 
@@ -265,7 +291,7 @@ def run_ours(args, rank, world, local_rank):
     n = H * S * d
     host = {t: torch.empty(n, dtype=torch.int16, pin_memory=True) for t in ("q", "k", "v")}
     for i, t in enumerate(("q", "k", "v")):
-        inputs.tensor(cfg, i, out=host[t].numpy().view(np.uint16), seed=seed)
+        inputs.tensor(cfg, i, h0=h0, nh=H, out=host[t].numpy().view(np.uint16), seed=seed)
     seg_h = torch.from_numpy(seg).pin_memory()
     times_h = torch.from_numpy(times).pin_memory()
     o_h = torch.empty(n, dtype=torch.int16, pin_memory=True)
@@ -356,24 +382,32 @@ def run_ours(args, rank, world, local_rank):
         if h3.check(ws) != h3.OK:
             raise RuntimeError("device status after e2e")
 
-    # max over ranks
+    # max over ranks; with head sharding the job's work is the sum of the ranks' shares
     ms, e2e_ms, fwd_ms, route_ms = max_over_ranks([ms, e2e_ms, fwd_ms, route_ms], world, dev)
+    local_flops, local_mma = eff_flops, mma_pairs
+    if sharded:
+        eff_flops, mma_pairs = sum_over_ranks([eff_flops, mma_pairs], world, dev)
 
     if rank != 0:
         return
     peaks, peak_kind = measured_peaks()
     ms_step = ms / args.steps
-    value = whole_job_tflops(eff_flops, args.steps, world, ms)
-    e2e_value = whole_job_tflops(eff_flops, args.steps, world, e2e_ms)
-    attn_tflops = eff_flops / (fwd_ms * 1e-3) / 1e12
+    # whole job: weak scaling = world independent calls; sharded = one call split over the ranks
+    job_world = 1 if sharded else world
+    value = whole_job_tflops(eff_flops, args.steps, job_world, ms)
+    e2e_value = whole_job_tflops(eff_flops, args.steps, job_world, e2e_ms)
+    attn_tflops = (local_flops if sharded else eff_flops) / (fwd_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     route_bytes = 2 * H * p.n_video_blocks * 64 * d * 2  # Q and K video rows, read once by the pool
     line = {
         "metric": "effective attention TFLOP/s (S=116883, H=56, d=128, sparsity 0.90, penalty on)",
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "strong" if sharded else "weak",
+        "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded counter-based generator, cluster-mean Q/K)",
-        "config": {"workload": WORKLOAD, "H": H, "S": S, "d": d, "block": 64, "sparsity": sparsity,
+        "config": {"workload": WORKLOAD, "H": cfg.H, "S": S, "d": d, "block": 64, "sparsity": sparsity,
+                   "parallelism": (f"head-sharded over {world} GPUs (rank 0: heads {h0}..{h0 + H - 1})" if sharded
+                                   else f"{world} independent calls, one per GPU"),
                    "k": int(p.k), "seed": seed, "l2": "no flush: Q+K+V = 5.0 GB per step, far above the 126 MB L2",
                    "effective_tflop_per_call": eff_flops / 1e12,
                    "executed_mma_tflop_per_call": 4 * d * mma_pairs / 1e12,
@@ -415,6 +449,9 @@ def main():
     ap.add_argument("--heads", type=int, default=None,
                     help="run the same packing with fewer heads (profiling captures only; the default is 56)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--shard", choices=["none", "heads"], default="none",
+                    help="N>1: 'none' = one independent call per GPU (weak scaling); 'heads' = one call, its heads "
+                         "split over the GPUs (strong scaling)")
     ap.add_argument("--chunk-heads", type=int, default=2, help="heads per pipelined chunk of the host-buffer call")
     args = ap.parse_args()
     if args.warmup < 3:
