@@ -382,8 +382,27 @@ def run_ours(args, rank, world, local_rank):
         if h3.check(ws) != h3.OK:
             raise RuntimeError("device status after e2e")
 
+    # partition merge (h3attn_merge) at full size: two partitions of this call's O/LSE shape, HBM-bound
+    merge_ms = float("nan")
+    if not args.no_merge:
+        lse_a = torch.zeros((H, S), dtype=torch.float32, device=dev)
+        lse_b = torch.full((H, S), -0.5, dtype=torch.float32, device=dev)
+        o2 = torch.empty_like(o)
+        l2 = torch.empty_like(lse_a)
+        for _ in range(3):
+            h3.merge([o, qd], [lse_a, lse_b], out=o2, lse=l2)
+        m0 = torch.cuda.Event(enable_timing=True)
+        m1 = torch.cuda.Event(enable_timing=True)
+        m0.record(stream)
+        for _ in range(args.steps):
+            h3.merge([o, qd], [lse_a, lse_b], out=o2, lse=l2)
+        m1.record(stream)
+        torch.cuda.synchronize(dev)
+        merge_ms = m0.elapsed_time(m1) / args.steps
+        del lse_a, lse_b, o2, l2
+
     # max over ranks; with head sharding the job's work is the sum of the ranks' shares
-    ms, e2e_ms, fwd_ms, route_ms = max_over_ranks([ms, e2e_ms, fwd_ms, route_ms], world, dev)
+    ms, e2e_ms, fwd_ms, route_ms, merge_ms = max_over_ranks([ms, e2e_ms, fwd_ms, route_ms, merge_ms], world, dev)
     local_flops, local_mma = eff_flops, mma_pairs
     if sharded:
         eff_flops, mma_pairs = sum_over_ranks([eff_flops, mma_pairs], world, dev)
@@ -419,6 +438,10 @@ def run_ours(args, rank, world, local_rank):
                      "peak_source": f"{peak_kind} bf16_tflops_sustained"},
         "routing": {"ms": route_ms, "bytes_read": route_bytes, "gbs": route_bytes / (route_ms * 1e-3) / 1e9,
                     "hbm_peak_gbs": peaks["hbm_gbs"]},
+        "merge": None if args.no_merge else {
+            "kernel": "merge_kernel (h3attn_merge: two partitions, O bf16 [H][S][d] + LSE f32, out O + LSE)",
+            "ms": merge_ms, "bytes": 3 * H * S * (d * 2 + 4),
+            "gbs": 3 * H * S * (d * 2 + 4) / (merge_ms * 1e-3) / 1e9, "hbm_peak_gbs": peaks["hbm_gbs"]},
         "gpu_launches": 5 * args.steps,  # pool_split, score_gemm, topk, kv_desc, attn
         "clocks": clk,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -449,6 +472,7 @@ def main():
     ap.add_argument("--heads", type=int, default=None,
                     help="run the same packing with fewer heads (profiling captures only; the default is 56)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--no-merge", action="store_true", help="skip the partition-merge measurement")
     ap.add_argument("--shard", choices=["none", "heads"], default="none",
                     help="N>1: 'none' = one independent call per GPU (weak scaling); 'heads' = one call, its heads "
                          "split over the GPUs (strong scaling)")

@@ -26,7 +26,7 @@ SEG_TEXT, SEG_IMAGE_REF, SEG_AUDIO, SEG_GUIDE, SEG_OUTPUT = 0, 1, 2, 3, 4
 EXPORTS = ("h3attn_plan_init", "h3attn_workspace_bytes", "h3attn_pool", "h3attn_route", "h3attn_route_static",
            "h3attn_forward",
            "h3attn_dense_workspace_bytes", "h3attn_dense_biased", "h3attn_check", "h3attn_selftest_timeout",
-           "h3attn_attend_host", "h3attn_strerror")
+           "h3attn_attend_host", "h3attn_merge", "h3attn_strerror")
 
 
 class H3Error(RuntimeError):
@@ -88,6 +88,9 @@ def lib():
         L.h3attn_attend_host.argtypes = [PP, _P, _P, _P, _P, _P, ctypes.POINTER(Penalty), _P, _P, _P, _P, _P, _P,
                                          _P, _P, _P, _P, _P, ctypes.c_size_t, ctypes.c_int, _P, _P, _P]
         L.h3attn_attend_host.restype = ctypes.c_int
+        L.h3attn_merge.argtypes = [ctypes.c_int, ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(ctypes.c_float),
+                                   ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P]
+        L.h3attn_merge.restype = ctypes.c_int
         L.h3attn_check.argtypes = [_P, _P]
         L.h3attn_check.restype = ctypes.c_int
         L.h3attn_selftest_timeout.argtypes = [_P, ctypes.c_uint32, _P]
@@ -228,6 +231,27 @@ def attend_host(p: Plan, q_host, k_host, v_host, seg_host, times_host, o_host, *
         q.data_ptr(), k.data_ptr(), v.data_ptr(), seg.data_ptr(), _dptr(times), _dptr(kv_sel), o.data_ptr(),
         _dptr(lse), ws.data_ptr(), ws.numel(), chunk_heads, _stream(stream), _stream(copy_in_stream),
         _stream(copy_out_stream)), "attend_host")
+
+
+def merge(o_parts, lse_parts, log_w=None, out=None, lse: bool | torch.Tensor = False, stream=None):
+    """Merge normalised partition results (forward outputs o [H, S, d] bf16 and lse [H, S] float32 over key
+    sets) with multipliers exp(log_w[i]); returns (O, LSE or None)."""
+    n = len(o_parts)
+    if n != len(lse_parts) or n == 0:
+        raise ValueError("o_parts and lse_parts must be non-empty and of equal length")
+    _check_qkv(*o_parts)
+    H, S, d = o_parts[0].shape
+    for t in lse_parts:
+        if not (t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and tuple(t.shape) == (H, S)):
+            raise ValueError("lse parts must be contiguous CUDA float32 [H, S]")
+    o = torch.empty_like(o_parts[0]) if out is None else out
+    lse_t = lse if isinstance(lse, torch.Tensor) else (
+        torch.empty((H, S), dtype=torch.float32, device=o.device) if lse else None)
+    op = (_P * n)(*[t.data_ptr() for t in o_parts])
+    lp = (_P * n)(*[t.data_ptr() for t in lse_parts])
+    lw = None if log_w is None else (ctypes.c_float * n)(*[float(x) for x in log_w])
+    _raise(lib().h3attn_merge(n, op, lp, lw, H, S, d, o.data_ptr(), _dptr(lse_t), _stream(stream)), "merge")
+    return o, lse_t
 
 
 def check(ws: torch.Tensor, stream=None) -> int:

@@ -324,6 +324,31 @@ int h3attn_attend_host(const h3attn_plan* plan, const uint16_t* q_host, const ui
   return rc;
 }
 
+int h3attn_merge(int n_parts, const uint16_t* const* o_parts, const float* const* lse_parts, const float* log_w,
+                 int H, int S, int d, uint16_t* o, float* lse, void* stream) {
+  if (n_parts < 1 || n_parts > h3::kMaxMergeParts || o_parts == nullptr || lse_parts == nullptr || o == nullptr)
+    return H3ATTN_EINVAL;
+  if (H <= 0 || S <= 0) return H3ATTN_EINVAL;
+  if (!(d == 64 || d == 128)) return H3ATTN_EUNSUPPORTED;
+  h3::MergeParts parts{};
+  parts.n = n_parts;
+  for (int i = 0; i < n_parts; ++i) {
+    if (o_parts[i] == nullptr || lse_parts[i] == nullptr) return H3ATTN_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(o_parts[i]) & 15u) || (reinterpret_cast<uintptr_t>(lse_parts[i]) & 3u))
+      return H3ATTN_EALIGN;
+    const float lw = log_w != nullptr ? log_w[i] : 0.0f;
+    if (std::isnan(lw) || lw == INFINITY) return H3ATTN_EINVAL;
+    parts.o[i] = o_parts[i];
+    parts.lse[i] = lse_parts[i];
+    parts.log_w[i] = lw;
+  }
+  if ((reinterpret_cast<uintptr_t>(o) & 15u) || (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return H3ATTN_EALIGN;
+  if (h3::launch_merge(parts, (long long)H * S, d, o, lse, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return H3ATTN_ECUDA;
+  return H3ATTN_OK;
+}
+
 size_t h3attn_dense_workspace_bytes(int S) {
   if (S <= 0) return 0;
   const int n_blocks = (S + h3::kBlock - 1) / h3::kBlock;

@@ -74,6 +74,17 @@ cudaError_t launch_route_pipeline(const uint16_t* q, const uint16_t* k, int32_t*
                                   int first_video_block, int n_video, int kk, void* scratch, int* status,
                                   cudaStream_t stream);
 
+// partition merge (h3attn_merge): up to kMaxMergeParts partitions, passed by value
+constexpr int kMaxMergeParts = 8;
+struct MergeParts {
+  const uint16_t* o[kMaxMergeParts];  // bf16 [rows][d]
+  const float* lse[kMaxMergeParts];   // [rows]
+  float log_w[kMaxMergeParts];
+  int n;
+};
+cudaError_t launch_merge(const MergeParts& parts, long long rows, int d, uint16_t* o, float* lse,
+                         cudaStream_t stream);
+
 cudaError_t launch_selftest_timeout(int* status, uint32_t polls, cudaStream_t stream);
 
 }  // namespace h3

@@ -208,6 +208,25 @@ H3ATTN_API int h3attn_attend_host(const h3attn_plan* plan, const uint16_t* q_hos
                                   float* lse, void* ws, size_t ws_bytes, int chunk_heads, void* stream,
                                   void* copy_in_stream, void* copy_out_stream);
 
+/* Merge of normalised partition results ("Flash Partitions for H3 native
+ * temporal alignment", section 4 "Why log-sum-exp is necessary"): partition i
+ * is an attention output O_i over some key set (normalised by its own sum)
+ * with its natural-log normaliser L_i -- h3attn_forward's o and lse -- and a
+ * non-negative multiplier w_i of its probabilities, given as log_w[i] (-inf
+ * for w_i = 0; log_w NULL: every w_i = 1).  Per (head, row):
+ *     adjusted_L_i = L_i + log w_i,  L = logsumexp_i adjusted_L_i,
+ *     O = sum_i exp(adjusted_L_i - L) O_i    (fp32, rounded to bf16 RNE),
+ * which for disjoint key sets equals the attention over their union with
+ * each set's probabilities scaled by its w_i.  A row whose adjusted
+ * normalisers are all -inf gets O = 0 and L = -inf.
+ *  n_parts in [1, 8]; o_parts / lse_parts: host arrays of n_parts device
+ *  pointers to bf16 [H][S][d] (16-byte aligned) and float32 [H][S]; log_w:
+ *  host array of n_parts floats (no NaN, no +inf) or NULL; o: bf16 [H][S][d]
+ *  device, 16-byte aligned (may be o_parts[0]); lse: float32 [H][S] device or
+ *  NULL. */
+H3ATTN_API int h3attn_merge(int n_parts, const uint16_t* const* o_parts, const float* const* lse_parts,
+                            const float* log_w, int H, int S, int d, uint16_t* o, float* lse, void* stream);
+
 /* Dense biased attention (every query attends every key; the penalty on
  * output -> guide pairs): h3attn_forward with a dense plan and kv_sel NULL.
  * Needs h3attn_dense_workspace_bytes(S) bytes of zero-filled workspace (the

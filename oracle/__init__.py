@@ -57,6 +57,8 @@ def lib():
         L.oracle_attend.restype = None
         L.oracle_attend_partitions.argtypes = attend_args
         L.oracle_attend_partitions.restype = None
+        L.oracle_merge.argtypes = [ctypes.c_int, ctypes.c_long, ctypes.c_int, _P, _P, _P, _P, _P]
+        L.oracle_merge.restype = None
         L.oracle_threads.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -167,3 +169,18 @@ def attend_partitions(q, k, v, seg, times, pen=None, sel=None, heads=None, rows=
         heads = np.repeat(np.arange(H), S)
         rows = np.tile(np.arange(S), H)
     return _attend(lib().oracle_attend_partitions, q, k, v, seg, times, pen, sel, heads, rows, B)
+
+
+def merge(o_parts, lse_parts, log_w=None):
+    """Flash-Partitions merge of normalised partition results ("Flash Partitions for H3 native temporal
+    alignment", section 4): o_parts [n][rows][d], lse_parts [n][rows] (natural log), log_w [n] or None
+    (every multiplier 1).  Returns (O [rows][d], L [rows]) in fp64."""
+    o = np.ascontiguousarray(o_parts, dtype=np.float64)
+    l = np.ascontiguousarray(lse_parts, dtype=np.float64)
+    n, rows, d = o.shape
+    assert l.shape == (n, rows)
+    lw = None if log_w is None else np.ascontiguousarray(log_w, dtype=np.float64)
+    out = np.empty((rows, d), np.float64)
+    out_l = np.empty(rows, np.float64)
+    lib().oracle_merge(n, rows, d, o.ctypes.data, l.ctypes.data, _ptr(lw), out.ctypes.data, out_l.ctypes.data)
+    return out, out_l

@@ -437,3 +437,40 @@ void oracle_attend_partitions(int H, int S, int d, int B, const uint8_t *seg,
     free(vid_index);
     free(nonvideo);
 }
+
+/*
+ * Merge of normalised partition results ([FP §4] "Why log-sum-exp is
+ * necessary"): partition i has output O_i (already divided by its own
+ * normaliser), natural-log normaliser L_i and a non-negative multiplier w_i
+ * given as log_w[i] (-inf for w_i = 0; log_w NULL means every w_i = 1).
+ *     adjusted_L_i = L_i + log w_i
+ *     L            = logsumexp_i adjusted_L_i
+ *     O            = sum_i exp(adjusted_L_i - L) O_i
+ * A row whose adjusted normalisers are all -inf gets O = 0 and L = -inf.
+ * o_parts [n_parts][rows][d], lse_parts [n_parts][rows]; o [rows][d], lse [rows].
+ */
+void oracle_merge(int n_parts, long rows, int d, const double *o_parts, const double *lse_parts,
+                  const double *log_w, double *o, double *lse) {
+    for (long r = 0; r < rows; ++r) {
+        double m = -INFINITY;
+        for (int i = 0; i < n_parts; ++i) {
+            double a = lse_parts[(long)i * rows + r] + (log_w ? log_w[i] : 0.0);
+            if (a > m) m = a;
+        }
+        double *orow = o + r * d;
+        for (int c = 0; c < d; ++c) orow[c] = 0.0;
+        if (m == -INFINITY) {
+            lse[r] = -INFINITY;
+            continue;
+        }
+        double s = 0.0;
+        for (int i = 0; i < n_parts; ++i) s += exp(lse_parts[(long)i * rows + r] + (log_w ? log_w[i] : 0.0) - m);
+        double L = m + log(s);
+        for (int i = 0; i < n_parts; ++i) {
+            double w = exp(lse_parts[(long)i * rows + r] + (log_w ? log_w[i] : 0.0) - L);
+            const double *oi = o_parts + ((long)i * rows + r) * d;
+            for (int c = 0; c < d; ++c) orow[c] += w * oi[c];
+        }
+        lse[r] = L;
+    }
+}

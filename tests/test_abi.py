@@ -125,6 +125,13 @@ def test_host_validation_before_any_device_work():
                                 None) == h3.EINVAL  # chunk_heads > H
     assert L.h3attn_attend_host(ctypes.byref(p), *args[:5], None, *args[5:16], 16, 1, None, None,
                                 None) == h3.EWORKSPACE
+    # partition merge: counts, pointers, d
+    ptrs = (ctypes.c_void_p * 9)(*([fake] * 9))
+    assert L.h3attn_merge(0, ptrs, ptrs, None, 1, 64, 128, fake, None, None) == h3.EINVAL
+    assert L.h3attn_merge(9, ptrs, ptrs, None, 1, 64, 128, fake, None, None) == h3.EINVAL
+    assert L.h3attn_merge(2, ptrs, ptrs, None, 1, 64, 96, fake, None, None) == h3.EUNSUPPORTED
+    bad_w = (ctypes.c_float * 2)(0.0, float("nan"))
+    assert L.h3attn_merge(2, ptrs, ptrs, bad_w, 1, 64, 128, fake, None, None) == h3.EINVAL
     p.k = 0  # corrupt plan
     assert L.h3attn_workspace_bytes(ctypes.byref(p)) == 0
     for code in [0, -1, -2, -3, -4, -5, -6, -7, -99]:

@@ -294,3 +294,58 @@ def test_sampled_rows_equal_full_rows():
     o2, l2 = oracle.attend(q, k, v, seg, times, pen=DEF, heads=heads, rows=rows)
     assert np.array_equal(o2, o.reshape(H, S, d)[heads, rows])
     assert np.array_equal(l2, lse.reshape(H, S)[heads, rows])
+
+
+# ------------------------------------------------------------------ partition merge
+# "Flash Partitions for H3 native temporal alignment", section 4: normalised partition outputs
+# O_i with log normalisers L_i and multipliers w_i merge through logsumexp of L_i + log w_i.
+# Pinned against brute-force softmax over disjoint key sets (numpy, fp64), not against the
+# oracle's own partition path.
+
+def _brute_partitions(x, v, groups, w=None):
+    """x [rows][n_keys] scores, v [n_keys][d]; groups: disjoint key index lists.
+    Returns per-group (O_g, L_g) and the weighted softmax over all keys."""
+    parts_o, parts_l = [], []
+    for g in groups:
+        e = np.exp(x[:, g])
+        parts_l.append(np.log(e.sum(axis=1)))
+        parts_o.append(e @ v[g] / e.sum(axis=1, keepdims=True))
+    mult = np.ones(x.shape[1])
+    if w is not None:
+        for g, wg in zip(groups, w):
+            mult[g] = wg
+    e = np.exp(x) * mult[None, :]
+    return np.array(parts_o), np.array(parts_l), e @ v / e.sum(axis=1, keepdims=True), np.log(e.sum(axis=1))
+
+
+def test_merge_of_disjoint_partitions_is_the_softmax_over_their_union():
+    rng = np.random.default_rng(5)
+    x = rng.normal(0, 3, size=(7, 40))
+    v = rng.normal(size=(40, 5))
+    groups = [list(range(0, 9)), list(range(9, 30)), list(range(30, 40))]
+    po, pl, want_o, want_l = _brute_partitions(x, v, groups)
+    o, l = oracle.merge(po, pl)
+    assert np.abs(o - want_o).max() < 1e-12 and np.abs(l - want_l).max() < 1e-12
+
+
+def test_merge_weights_scale_each_partitions_probabilities():
+    rng = np.random.default_rng(6)
+    x = rng.normal(0, 2, size=(5, 24))
+    v = rng.normal(size=(24, 3))
+    groups = [list(range(0, 10)), list(range(10, 24))]
+    w = [0.25, 1.7]
+    po, pl, want_o, want_l = _brute_partitions(x, v, groups, w)
+    o, l = oracle.merge(po, pl, np.log(w))
+    assert np.abs(o - want_o).max() < 1e-12 and np.abs(l - want_l).max() < 1e-12
+
+
+def test_merge_special_cases():
+    rng = np.random.default_rng(7)
+    po = rng.normal(size=(2, 4, 3))
+    pl = rng.normal(size=(2, 4))
+    o, l = oracle.merge(po[:1], pl[:1])                         # one partition, weight 1: unchanged
+    assert np.array_equal(o, po[0]) and np.allclose(l, pl[0], atol=0, rtol=0)
+    o, l = oracle.merge(po, pl, np.array([0.0, -np.inf]))       # weight 0 drops a partition
+    assert np.allclose(o, po[0], atol=1e-15) and np.allclose(l, pl[0], atol=1e-15)
+    o, l = oracle.merge(po, np.full((2, 4), -np.inf))           # nothing attended
+    assert np.all(o == 0) and np.all(l == -np.inf)
