@@ -59,6 +59,8 @@ def lib():
         L.oracle_attend_partitions.restype = None
         L.oracle_merge.argtypes = [ctypes.c_int, ctypes.c_long, ctypes.c_int, _P, _P, _P, _P, _P]
         L.oracle_merge.restype = None
+        L.oracle_tail.argtypes = [ctypes.c_int] * 4 + [_P] * 5 + [ctypes.c_int, _P, _P]
+        L.oracle_tail.restype = None
         L.oracle_threads.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -184,3 +186,35 @@ def merge(o_parts, lse_parts, log_w=None):
     out_l = np.empty(rows, np.float64)
     lib().oracle_merge(n, rows, d, o.ctypes.data, l.ctypes.data, _ptr(lw), out.ctypes.data, out_l.ctypes.data)
     return out, out_l
+
+
+def tail(q, k, v, seg, sel, B: int = 64):
+    """Pooled tail term per (head, video query block) ("H3 SLA Attention", inputs table, tail_correction):
+    the routed-out video key blocks as one partition, each block counted as its valid rows at its pooled
+    score with its mean value.  sel: routed lists [H][nV][k].  Returns (Lt [H][nV], Ot [H][nV][d]) fp64."""
+    H, S, d = np.shape(q)
+    sel = np.ascontiguousarray(sel, dtype=np.int32)
+    nv, kk = sel.shape[1], sel.shape[2]
+    lt = np.empty((H, nv), np.float64)
+    ot = np.empty((H, nv, d), np.float64)
+    seg_c, q_c, k_c, v_c = _c(seg, np.uint8), _c(q, np.uint16), _c(k, np.uint16), _c(v, np.uint16)
+    lib().oracle_tail(H, S, d, B, seg_c.ctypes.data, q_c.ctypes.data, k_c.ctypes.data, v_c.ctypes.data,
+                      sel.ctypes.data, kk, lt.ctypes.data, ot.ctypes.data)
+    return lt, ot
+
+
+def attend_tail(q, k, v, seg, times, pen, sel, heads, rows, B: int = 64):
+    """Routed attention with the pooled tail term merged in, for (head, row) pairs: rows of video query
+    blocks merge their exact routed result with their block's tail partition; other rows are unchanged."""
+    o, l = attend(q, k, v, seg, times, pen=pen, sel=sel, heads=heads, rows=rows, B=B)
+    lt, ot = tail(q, k, v, seg, sel, B=B)
+    fvb = int(block_classes(seg, B).sum())
+    blk = np.asarray(rows) // B - fvb
+    video = blk >= 0
+    o2, l2 = o.copy(), l.copy()
+    if video.any():
+        hh = np.asarray(heads)[video]
+        bb = blk[video]
+        mo, ml = merge(np.stack([o[video], ot[hh, bb]]), np.stack([l[video], lt[hh, bb]]))
+        o2[video], l2[video] = mo, ml
+    return o2, l2

@@ -474,3 +474,77 @@ void oracle_merge(int n_parts, long rows, int d, const double *o_parts, const do
         lse[r] = L;
     }
 }
+
+/*
+ * Pooled tail term ("H3 SLA Attention", inputs table, tail_correction):
+ * instead of dropping the video key blocks top-k left out, one pooled term
+ * stands in for all of them, scored from the pooled centroids the selection
+ * already uses.  Reading (the page gives no formula): for video query block i
+ * of head h, with D_i the video key blocks not in its routed list, n_j the
+ * valid rows of block j and Qp, Kp, Vp the block means,
+ *     Lt_i = log sum_{j in D_i} n_j exp(Qp_i . Kp_j / sqrt(d)),
+ *     Ot_i = sum_{j in D_i} n_j exp(Qp_i . Kp_j / sqrt(d) - Lt_i) Vp_j,
+ * i.e. each dropped block counts as n_j keys at its pooled score with its mean
+ * value, without the temporal penalty (routing does not see it either).  Each
+ * row of block i then merges (Ot_i, Lt_i) with its exact routed attention as a
+ * partition of weight 1 (oracle_merge).  D_i empty: Lt_i = -inf.
+ * sel [H][nV][k] absolute block ids; lt [H][nV]; ot [H][nV][d].
+ */
+void oracle_tail(int H, int S, int d, int B, const uint8_t *seg, const uint16_t *q, const uint16_t *k,
+                 const uint16_t *v, const int32_t *sel, int kk, double *lt, double *ot) {
+    int nkb = (S + B - 1) / B;
+    uint8_t *nonvideo = (uint8_t *)calloc((size_t)nkb, 1);
+    oracle_block_classes(S, B, seg, nonvideo);
+    int fvb = 0;
+    while (fvb < nkb && nonvideo[fvb]) ++fvb;
+    int nv = nkb - fvb;
+    double *qp = (double *)malloc(sizeof(double) * (size_t)H * nkb * d);
+    double *kp = (double *)malloc(sizeof(double) * (size_t)H * nkb * d);
+    double *vp = (double *)malloc(sizeof(double) * (size_t)H * nkb * d);
+    oracle_pool(H, S, d, B, q, qp);
+    oracle_pool(H, S, d, B, k, kp);
+    oracle_pool(H, S, d, B, v, vp);
+    double inv_sqrt_d = 1.0 / sqrt((double)d);
+#pragma omp parallel for schedule(dynamic)
+    for (long hi = 0; hi < (long)H * nv; ++hi) {
+        int h = (int)(hi / nv), i = (int)(hi % nv);
+        uint8_t *kept = (uint8_t *)calloc((size_t)nkb, 1);
+        for (int t = 0; t < kk; ++t) kept[sel[(size_t)hi * kk + t]] = 1;
+        const double *qrow = qp + ((size_t)h * nkb + fvb + i) * d;
+        double m = -INFINITY;
+        double *x = (double *)malloc(sizeof(double) * (size_t)nkb);
+        for (int j = fvb; j < nkb; ++j) {
+            x[j] = -INFINITY;
+            if (kept[j]) continue;
+            const double *krow = kp + ((size_t)h * nkb + j) * d;
+            double s = 0.0;
+            for (int c = 0; c < d; ++c) s += qrow[c] * krow[c];
+            int nj = (j + 1) * B <= S ? B : S - j * B;
+            x[j] = s * inv_sqrt_d + log((double)nj);
+            if (x[j] > m) m = x[j];
+        }
+        double *o = ot + (size_t)hi * d;
+        for (int c = 0; c < d; ++c) o[c] = 0.0;
+        if (m == -INFINITY) {
+            lt[hi] = -INFINITY;
+        } else {
+            double sum = 0.0;
+            for (int j = fvb; j < nkb; ++j)
+                if (x[j] > -INFINITY) sum += exp(x[j] - m);
+            double L = m + log(sum);
+            for (int j = fvb; j < nkb; ++j) {
+                if (x[j] == -INFINITY) continue;
+                double w = exp(x[j] - L);
+                const double *vrow = vp + ((size_t)h * nkb + j) * d;
+                for (int c = 0; c < d; ++c) o[c] += w * vrow[c];
+            }
+            lt[hi] = L;
+        }
+        free(x);
+        free(kept);
+    }
+    free(qp);
+    free(kp);
+    free(vp);
+    free(nonvideo);
+}

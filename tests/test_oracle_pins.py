@@ -349,3 +349,50 @@ def test_merge_special_cases():
     assert np.allclose(o, po[0], atol=1e-15) and np.allclose(l, pl[0], atol=1e-15)
     o, l = oracle.merge(po, np.full((2, 4), -np.inf))           # nothing attended
     assert np.all(o == 0) and np.all(l == -np.inf)
+
+
+# ------------------------------------------------------------------ pooled tail term
+# "H3 SLA Attention", inputs table, tail_correction: the routed-out key blocks enter through one pooled
+# term.  When every 64-row block consists of identical rows, a block's pooled score and mean value are
+# exact for each of its rows, so routed attention with the tail term must equal dense attention.
+
+def _blockwise_constant(cfg):
+    """Q, K, V of cfg with every row replaced by its block's first row (bf16 bits)."""
+    out = []
+    for t in range(3):
+        x = inputs.tensor(cfg, t).copy()
+        H, S, d = x.shape
+        for b in range(0, S, 64):
+            x[:, b:b + 64] = x[:, b:b + 1]
+        out.append(x)
+    return out
+
+
+def test_tail_term_is_exact_for_blockwise_constant_inputs():
+    segs = [inputs.Segment(inputs.SEG_TEXT, 64), inputs.Segment(inputs.SEG_AUDIO, 64),
+            inputs.Segment(inputs.SEG_OUTPUT, 8 * 64, 8)]
+    cfg = inputs.custom(2, 32, segs, seed=3, cluster_norm=2.0)
+    seg, times, _ = cfg.layout()
+    q, k, v = _blockwise_constant(cfg)
+    sel, _, _ = oracle.route(q, k, seg, 0.75)
+    H, S = 2, cfg.S
+    heads, rows = np.repeat(np.arange(H), S), np.tile(np.arange(S), H)
+    dense_o, dense_l = oracle.attend(q, k, v, seg, times, pen=None, sel=None, heads=heads, rows=rows)
+    routed_o, _ = oracle.attend(q, k, v, seg, times, pen=None, sel=sel, heads=heads, rows=rows)
+    tail_o, tail_l = oracle.attend_tail(q, k, v, seg, times, None, sel, heads, rows)
+    assert np.abs(routed_o - dense_o).max() > 1e-3            # routing alone drops mass
+    assert np.abs(tail_o - dense_o).max() < 1e-12 and np.abs(tail_l - dense_l).max() < 1e-12
+
+
+def test_tail_term_is_absent_without_dropped_blocks():
+    segs = [inputs.Segment(inputs.SEG_TEXT, 64), inputs.Segment(inputs.SEG_OUTPUT, 4 * 64, 4)]
+    cfg = inputs.custom(1, 32, segs, seed=4, cluster_norm=2.0)
+    seg, times, _ = cfg.layout()
+    q, k, v = (inputs.tensor(cfg, t) for t in range(3))
+    sel, _, _ = oracle.route(q, k, seg, 0.0)                  # every video block kept
+    lt, ot = oracle.tail(q, k, v, seg, sel)
+    assert np.all(lt == -np.inf) and np.all(ot == 0)
+    rows = np.arange(cfg.S)
+    a = oracle.attend(q, k, v, seg, times, pen=None, sel=sel, heads=np.zeros_like(rows), rows=rows)
+    b = oracle.attend_tail(q, k, v, seg, times, None, sel, np.zeros_like(rows), rows)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
