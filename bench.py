@@ -401,8 +401,30 @@ def run_ours(args, rank, world, local_rank):
         merge_ms = m0.elapsed_time(m1) / args.steps
         del lse_a, lse_b, o2, l2
 
+    # pooled tail term (h3attn_tail_correct) at full size: after route + forward with LSE on this call's
+    # inputs; its kernels read V's video rows, the pooled scores, the weights and the O/LSE of video rows
+    tail_ms = float("nan")
+    if not args.no_tail and p.n_video_blocks > 0:
+        lse_t = torch.empty((H, S), dtype=torch.float32, device=dev)
+        tail_ws = h3.tail_workspace(p, dev)
+        h3.route(p, qd, kd, ws, kv_sel=sel)
+        h3.forward(p, qd, kd, vd, seg_d, times_d, pen=pen, kv_sel=sel, ws=ws, out=o, lse=lse_t)
+        h3.tail_correct(p, vd, sel, o, lse_t, ws, tail_ws=tail_ws)
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            h3.tail_correct(p, vd, sel, o, lse_t, ws, tail_ws=tail_ws)
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        tail_ms = t0.elapsed_time(t1) / args.steps
+        if h3.check(ws) != h3.OK:
+            raise RuntimeError("device status after the tail correction")
+        del lse_t, tail_ws
+
     # max over ranks; with head sharding the job's work is the sum of the ranks' shares
-    ms, e2e_ms, fwd_ms, route_ms, merge_ms = max_over_ranks([ms, e2e_ms, fwd_ms, route_ms, merge_ms], world, dev)
+    ms, e2e_ms, fwd_ms, route_ms, merge_ms, tail_ms = max_over_ranks(
+        [ms, e2e_ms, fwd_ms, route_ms, merge_ms, tail_ms], world, dev)
     local_flops, local_mma = eff_flops, mma_pairs
     if sharded:
         eff_flops, mma_pairs = sum_over_ranks([eff_flops, mma_pairs], world, dev)
@@ -442,6 +464,9 @@ def run_ours(args, rank, world, local_rank):
             "kernel": "merge_kernel (h3attn_merge: two partitions, O bf16 [H][S][d] + LSE f32, out O + LSE)",
             "ms": merge_ms, "bytes": 3 * H * S * (d * 2 + 4),
             "gbs": 3 * H * S * (d * 2 + 4) / (merge_ms * 1e-3) / 1e9, "hbm_peak_gbs": peaks["hbm_gbs"]},
+        "tail": None if args.no_tail else {
+            "kernels": "pool_vt, tail_weights, tail_gemm (tcgen05), tail_merge (h3attn_tail_correct)",
+            "ms": tail_ms, "share_of_call": tail_ms / ms_step},
         "gpu_launches": 5 * args.steps,  # pool_split, score_gemm, topk, kv_desc, attn
         "clocks": clk,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -473,6 +498,7 @@ def main():
                     help="run the same packing with fewer heads (profiling captures only; the default is 56)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-merge", action="store_true", help="skip the partition-merge measurement")
+    ap.add_argument("--no-tail", action="store_true", help="skip the pooled-tail-term measurement")
     ap.add_argument("--shard", choices=["none", "heads"], default="none",
                     help="N>1: 'none' = one independent call per GPU (weak scaling); 'heads' = one call, its heads "
                          "split over the GPUs (strong scaling)")

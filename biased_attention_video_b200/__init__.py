@@ -26,7 +26,8 @@ SEG_TEXT, SEG_IMAGE_REF, SEG_AUDIO, SEG_GUIDE, SEG_OUTPUT = 0, 1, 2, 3, 4
 EXPORTS = ("h3attn_plan_init", "h3attn_workspace_bytes", "h3attn_pool", "h3attn_route", "h3attn_route_static",
            "h3attn_forward",
            "h3attn_dense_workspace_bytes", "h3attn_dense_biased", "h3attn_check", "h3attn_selftest_timeout",
-           "h3attn_attend_host", "h3attn_merge", "h3attn_strerror")
+           "h3attn_attend_host", "h3attn_merge", "h3attn_tail_workspace_bytes", "h3attn_tail_correct",
+           "h3attn_strerror")
 
 
 class H3Error(RuntimeError):
@@ -91,6 +92,10 @@ def lib():
         L.h3attn_merge.argtypes = [ctypes.c_int, ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(ctypes.c_float),
                                    ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P]
         L.h3attn_merge.restype = ctypes.c_int
+        L.h3attn_tail_workspace_bytes.argtypes = [PP]
+        L.h3attn_tail_workspace_bytes.restype = ctypes.c_size_t
+        L.h3attn_tail_correct.argtypes = [PP, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, ctypes.c_size_t, _P]
+        L.h3attn_tail_correct.restype = ctypes.c_int
         L.h3attn_check.argtypes = [_P, _P]
         L.h3attn_check.restype = ctypes.c_int
         L.h3attn_selftest_timeout.argtypes = [_P, ctypes.c_uint32, _P]
@@ -252,6 +257,23 @@ def merge(o_parts, lse_parts, log_w=None, out=None, lse: bool | torch.Tensor = F
     lw = None if log_w is None else (ctypes.c_float * n)(*[float(x) for x in log_w])
     _raise(lib().h3attn_merge(n, op, lp, lw, H, S, d, o.data_ptr(), _dptr(lse_t), _stream(stream)), "merge")
     return o, lse_t
+
+
+def tail_workspace(p: Plan, device="cuda") -> torch.Tensor:
+    n = lib().h3attn_tail_workspace_bytes(ctypes.byref(p))
+    if n == 0:
+        raise H3Error(EINVAL, "tail_workspace")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def tail_correct(p: Plan, v, kv_sel, o, lse, ws, tail_ws=None, stream=None) -> None:
+    """Fold the routed-out video key blocks into (o, lse) as one pooled term per query block, in place.
+    Call after route(p, q, k, ws, kv_sel) and forward(..., kv_sel, ws, out=o, lse=lse) with the same ws."""
+    _check_qkv(v, o)
+    tw = tail_workspace(p, v.device) if tail_ws is None else tail_ws
+    _raise(lib().h3attn_tail_correct(ctypes.byref(p), v.data_ptr(), kv_sel.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                     ws.data_ptr(), ws.numel(), tw.data_ptr(), tw.numel(), _stream(stream)),
+           "tail_correct")
 
 
 def check(ws: torch.Tensor, stream=None) -> int:

@@ -349,6 +349,33 @@ int h3attn_merge(int n_parts, const uint16_t* const* o_parts, const float* const
   return H3ATTN_OK;
 }
 
+size_t h3attn_tail_workspace_bytes(const h3attn_plan* plan) {
+  if (!plan_ok(plan) || plan->n_video_blocks == 0) return 0;
+  return h3::tail_scratch_layout(plan->H, plan->d, plan->n_video_blocks).total;
+}
+
+int h3attn_tail_correct(const h3attn_plan* plan, const uint16_t* v, const int32_t* kv_sel, uint16_t* o, float* lse,
+                        void* ws, size_t ws_bytes, void* tail_ws, size_t tail_ws_bytes, void* stream) {
+  if (!plan_ok(plan) || plan->n_video_blocks == 0) return H3ATTN_EINVAL;
+  if (v == nullptr || kv_sel == nullptr || o == nullptr || lse == nullptr) return H3ATTN_EINVAL;
+  const WsLayout w = ws_layout(plan->H, plan->d, plan->n_blocks, plan->n_video_blocks);
+  if (ws == nullptr || ws_bytes < w.total) return H3ATTN_EWORKSPACE;
+  if (tail_ws == nullptr || tail_ws_bytes < h3attn_tail_workspace_bytes(plan)) return H3ATTN_EWORKSPACE;
+  if (!aligned16(v) || !aligned16(o) || !aligned16(tail_ws) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+      (reinterpret_cast<uintptr_t>(kv_sel) & 3u))
+    return H3ATTN_EALIGN;
+  const size_t bitmap_smem = (size_t)8 * ((plan->n_video_blocks + 31) / 32) * 4;
+  if (bitmap_smem > (size_t)kMaxSmem) return H3ATTN_EUNSUPPORTED;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  const h3::RouteScratch r = h3::route_scratch_layout(plan->H, plan->d, plan->n_video_blocks);
+  const float* scores = reinterpret_cast<const float*>(wsb + w.route + r.scores);
+  if (h3::launch_tail(v, scores, r.ldc, kv_sel, plan->k, plan->H, plan->S, plan->d, plan->first_video_block,
+                      plan->n_video_blocks, o, lse, tail_ws, reinterpret_cast<int*>(wsb),
+                      static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return H3ATTN_ECUDA;
+  return H3ATTN_OK;
+}
+
 size_t h3attn_dense_workspace_bytes(int S) {
   if (S <= 0) return 0;
   const int n_blocks = (S + h3::kBlock - 1) / h3::kBlock;

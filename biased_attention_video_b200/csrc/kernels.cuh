@@ -74,6 +74,19 @@ cudaError_t launch_route_pipeline(const uint16_t* q, const uint16_t* k, int32_t*
                                   int first_video_block, int n_video, int kk, void* scratch, int* status,
                                   cudaStream_t stream);
 
+// pooled tail term (h3attn_tail_correct): scratch byte offsets of the bf16
+// weights [H][n_video][ldk], the transposed pooled V [H][d][ldk], the tail
+// outputs [H][n_video][d] (bf16) and the per-block log mass and 1 / mass
+struct TailScratch {
+  size_t w, vpt, ot, lt, inv_sum, total, ldk;
+};
+TailScratch tail_scratch_layout(int H, int d, int n_video);
+// scores: the fp32 pooled scores [H][n_video][ldc] routing left; o / lse
+// updated in place for the rows of video query blocks
+cudaError_t launch_tail(const uint16_t* v, const float* scores, size_t ldc, const int32_t* kv_sel, int kk, int H,
+                        int S, int d, int first_block, int n_video, uint16_t* o, float* lse, void* scratch,
+                        int* status, cudaStream_t stream);
+
 // partition merge (h3attn_merge): up to kMaxMergeParts partitions, passed by value
 constexpr int kMaxMergeParts = 8;
 struct MergeParts {

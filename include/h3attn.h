@@ -208,6 +208,32 @@ H3ATTN_API int h3attn_attend_host(const h3attn_plan* plan, const uint16_t* q_hos
                                   float* lse, void* ws, size_t ws_bytes, int chunk_heads, void* stream,
                                   void* copy_in_stream, void* copy_out_stream);
 
+/* Pooled tail term ("H3 SLA Attention", inputs table, tail_correction):
+ * instead of dropping the video key blocks a query block's top-k left out,
+ * fold them in as one pooled term, scored from the pooled centroids routing
+ * computed.  For video query block i of head h (dropped set D_i, n_j valid
+ * rows of block j, Qp/Kp/Vp block means):
+ *     Lt_i = log sum_{j in D_i} n_j exp(Qp_i . Kp_j / sqrt(d)),
+ *     Ot_i = sum_{j in D_i} n_j exp(Qp_i . Kp_j / sqrt(d) - Lt_i) Vp_j,
+ * no temporal penalty (routing sees none); each row of block i then merges
+ * (Ot_i, Lt_i) with its routed result (o, lse) as one more partition of weight
+ * 1 (the merge of h3attn_merge), in place.  Rows of dense (prefix) query
+ * blocks are unchanged.  The dot products are the fp32-accurate pooled scores
+ * routing computed; the weights n_j exp(...) and Vp are rounded to bf16 for the
+ * tensor-core sum (fp32 accumulation).
+ * Contract: call after h3attn_route(plan, q, k, kv_sel, ws, ...) and
+ * h3attn_forward(plan, ..., kv_sel, o, lse, ws, ...) with the same plan, ws
+ * and kv_sel, before anything else reuses ws (this call reads the pooled
+ * scores h3attn_route left in it).  v: bf16 [H][S][d] device; kv_sel as for
+ * h3attn_forward; o, lse: that call's outputs (lse not NULL), updated in
+ * place; tail_ws: device scratch of h3attn_tail_workspace_bytes(plan) bytes
+ * (about 0.43 GB at S = 116,883, H = 56, d = 128; no zeroing needed).
+ * Routed indices outside the video blocks are ignored. */
+H3ATTN_API size_t h3attn_tail_workspace_bytes(const h3attn_plan* plan);
+H3ATTN_API int h3attn_tail_correct(const h3attn_plan* plan, const uint16_t* v, const int32_t* kv_sel, uint16_t* o,
+                                   float* lse, void* ws, size_t ws_bytes, void* tail_ws, size_t tail_ws_bytes,
+                                   void* stream);
+
 /* Merge of normalised partition results ("Flash Partitions for H3 native
  * temporal alignment", section 4 "Why log-sum-exp is necessary"): partition i
  * is an attention output O_i over some key set (normalised by its own sum)
