@@ -78,26 +78,41 @@ def effective_pairs(p, sel: np.ndarray | None) -> int:
 
 def executed_mma_pairs(p, sel: np.ndarray | None) -> int:
     """(query, key) pairs the tensor cores actually process: per 128-row tile, the union
-    of its two query blocks' key lists, rounded up to 128-key tiles."""
+    of its two query blocks' key lists, rounded up to 128-key tiles.  The tiles are the
+    kernel's: adjacent blocks over the dense prefix (rounded up to an even block), then
+    the video blocks paired within groups of 32 by greedy largest list overlap (ties to
+    the lowest pair), an odd block out alone."""
     nkb = p.n_blocks
-    n_tiles_q = (nkb + 1) // 2
+    full = (nkb + 1) // 2                     # 128-key tiles of a dense row block
     if sel is None:
-        return int(p.H) * n_tiles_q * 128 * ((nkb + 1) // 2) * 128
-    total = 0
-    fvb = p.first_video_block
-    for t in range(n_tiles_q):
-        a, b = 2 * t, 2 * t + 1
-        if a < fvb or (b < nkb and b < fvb):
-            total += p.H * ((nkb + 1) // 2)
-            continue
-        la = sel[:, a - fvb]
-        if b < nkb:
-            lb = sel[:, b - fvb]
-            for h in range(p.H):
-                u = np.union1d(la[h], lb[h]).size + fvb
-                total += (u + 1) // 2
-        else:
-            total += p.H * ((la.shape[1] + fvb + 1) // 2)
+        return int(p.H) * full * 128 * full * 128
+    fvb, H, kk = p.first_video_block, int(p.H), sel.shape[2]
+    n_dense = (fvb + 1) // 2
+    total = H * n_dense * full                # a dense block makes its tile dense
+    first = 2 * n_dense
+    nv = nkb - fvb
+    G = 32
+    iu = np.triu_indices(G, 1)
+    tie = ((31 - iu[0]) * 32 + (31 - iu[1])).astype(np.int64)
+    for g0 in range(first, nkb, G):
+        gs = min(G, nkb - g0)
+        bits = np.zeros((H, G, nv), np.float32)
+        hh, ii = np.meshgrid(np.arange(H), np.arange(gs), indexing="ij")
+        lst = sel[:, g0 - fvb:g0 - fvb + gs] - fvb                  # [H][gs][k]
+        bits[hh[..., None], ii[..., None], lst] = 1.0
+        ov = np.einsum("hav,hbv->hab", bits, bits).astype(np.int64)[:, iu[0], iu[1]]
+        alive = np.zeros((H, G), bool)
+        alive[:, :gs] = True
+        for _ in range(gs // 2):
+            ok = alive[:, iu[0]] & alive[:, iu[1]]
+            key = np.where(ok, ov * 1024 + tie[None, :], -1)
+            c = key.argmax(axis=1)
+            u = 2 * kk - ov[np.arange(H), c]
+            total += int(((u + fvb + 1) // 2).sum())
+            alive[np.arange(H), iu[0][c]] = False
+            alive[np.arange(H), iu[1][c]] = False
+        if gs % 2:
+            total += H * ((kk + fvb + 1) // 2)
     return int(total) * 128 * 128
 
 

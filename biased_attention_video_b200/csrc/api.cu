@@ -26,7 +26,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 struct WsLayout {
-  size_t desc, gtime, slow, route, total;
+  size_t desc, gtime, slow, pairs, route, total;
 };
 
 // Attention scratch after the status word: per-key-block descriptors, per-key
@@ -37,14 +37,24 @@ size_t attn_scratch_bytes(int n_blocks) {
          align_up((size_t)(n_blocks + 31) / 32 * sizeof(uint32_t));
 }
 
-// status word | per-key-block descriptors | per-key guide times | routing scratch
-WsLayout ws_layout(int H, int d, int n_blocks, int n_video) {
+// query-block pair table of a routed call: one word per paired tile and head
+size_t pair_bytes(const h3attn_plan* plan) {
+  return plan->n_video_blocks > 0
+             ? align_up((size_t)plan->H * h3::paired_tiles(plan->n_blocks, plan->first_video_block) * sizeof(uint32_t))
+             : 0;
+}
+
+// status word | per-key-block descriptors | per-key guide times | slow-block
+// bitmap | query-block pairs | routing scratch
+WsLayout ws_layout(const h3attn_plan* plan) {
   WsLayout w;
   w.desc = kStatusBytes;
-  w.gtime = w.desc + align_up((size_t)n_blocks * sizeof(uint4));
-  w.slow = w.gtime + align_up((size_t)n_blocks * h3::kBlock * sizeof(float));
-  w.route = kStatusBytes + attn_scratch_bytes(n_blocks);
-  w.total = w.route + (n_video > 0 ? h3::route_scratch_layout(H, d, n_video).total : 0);
+  w.gtime = w.desc + align_up((size_t)plan->n_blocks * sizeof(uint4));
+  w.slow = w.gtime + align_up((size_t)plan->n_blocks * h3::kBlock * sizeof(float));
+  w.pairs = kStatusBytes + attn_scratch_bytes(plan->n_blocks);
+  w.route = w.pairs + pair_bytes(plan);
+  w.total = w.route +
+            (plan->n_video_blocks > 0 ? h3::route_scratch_layout(plan->H, plan->d, plan->n_video_blocks).total : 0);
   return w;
 }
 
@@ -114,7 +124,7 @@ int forward_impl(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, 
   p.lse = lse;
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   p.status = reinterpret_cast<int*>(wsb);
-  const WsLayout wl = ws_layout(plan->H, plan->d, plan->n_blocks, 0);
+  const WsLayout wl = ws_layout(plan);
   p.kv_desc = reinterpret_cast<const uint4*>(wsb + wl.desc);
   p.gtime = reinterpret_cast<const float*>(wsb + wl.gtime);
   p.slow_blocks = reinterpret_cast<const uint32_t*>(wsb + wl.slow);
@@ -129,7 +139,11 @@ int forward_impl(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, 
   }
   p.wait_polls = kWaitPolls;
   p.wait_ns = kWaitNs;
-  const int n_qtiles = (plan->n_blocks + 1) / 2;
+  // routed: adjacent pairs over the dense prefix, then the overlap pairing
+  p.qpairs = routed ? reinterpret_cast<const uint32_t*>(wsb + wl.pairs) : nullptr;
+  p.n_dense_tiles = routed ? h3::paired_first_block(plan->first_video_block) / 2 : (plan->n_blocks + 1) / 2;
+  p.n_paired_tiles = routed ? h3::paired_tiles(plan->n_blocks, plan->first_video_block) : 0;
+  const int n_qtiles = p.n_dense_tiles + p.n_paired_tiles;
 
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, q, plan->H, plan->S, plan->d) || !make_map(&tk, k, plan->H, plan->S, plan->d) ||
@@ -138,6 +152,9 @@ int forward_impl(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, 
   if (h3::launch_kv_desc(seg, pen_on ? times : nullptr, plan->S, plan->n_blocks, reinterpret_cast<uint4*>(wsb + wl.desc),
                          reinterpret_cast<float*>(wsb + wl.gtime), reinterpret_cast<uint32_t*>(wsb + wl.slow),
                          stream) != cudaSuccess)
+    return H3ATTN_ECUDA;
+  if (routed && h3::launch_pair(kv_sel, plan->H, plan->n_blocks, plan->first_video_block, plan->k,
+                                reinterpret_cast<uint32_t*>(wsb + wl.pairs), stream) != cudaSuccess)
     return H3ATTN_ECUDA;
   if (h3::launch_attn(tq, tk, tv, p, n_qtiles * plan->H, stream) != cudaSuccess) return H3ATTN_ECUDA;
   return H3ATTN_OK;
@@ -200,7 +217,7 @@ int h3attn_plan_init(h3attn_plan* plan, int H, int S, int d, int block, float sp
 
 size_t h3attn_workspace_bytes(const h3attn_plan* plan) {
   if (!plan_ok(plan)) return 0;
-  return ws_layout(plan->H, plan->d, plan->n_blocks, plan->n_video_blocks).total;
+  return ws_layout(plan).total;
 }
 
 int h3attn_pool(const h3attn_plan* plan, const uint16_t* x, int first_block, int n_out, float* out, void* stream) {
@@ -218,7 +235,7 @@ int h3attn_route(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, 
                  size_t ws_bytes, void* stream) {
   if (!plan_ok(plan) || q == nullptr || k == nullptr || kv_sel == nullptr) return H3ATTN_EINVAL;
   if (plan->n_video_blocks == 0) return H3ATTN_EINVAL;
-  const WsLayout w = ws_layout(plan->H, plan->d, plan->n_blocks, plan->n_video_blocks);
+  const WsLayout w = ws_layout(plan);
   if (ws == nullptr || ws_bytes < w.total) return H3ATTN_EWORKSPACE;
   if (!aligned16(q) || !aligned16(k) || !aligned16(ws) || (reinterpret_cast<uintptr_t>(kv_sel) & 3u))
     return H3ATTN_EALIGN;
@@ -235,7 +252,8 @@ int h3attn_forward(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k
                    const uint8_t* seg, const float* times, const h3attn_penalty* pen, const int32_t* kv_sel,
                    uint16_t* o, float* lse, void* ws, size_t ws_bytes, void* stream) {
   if (!plan_ok(plan)) return H3ATTN_EINVAL;
-  const size_t need = kStatusBytes + attn_scratch_bytes(plan->n_blocks);
+  // a routed call also needs the query-block pair table
+  const size_t need = kStatusBytes + attn_scratch_bytes(plan->n_blocks) + (kv_sel != nullptr ? pair_bytes(plan) : 0);
   if (kv_sel != nullptr && (reinterpret_cast<uintptr_t>(kv_sel) & 3u)) return H3ATTN_EALIGN;
   return forward_impl(plan, q, k, v, seg, times, pen, kv_sel, o, lse, ws, ws_bytes, need,
                       static_cast<cudaStream_t>(stream));
@@ -358,7 +376,7 @@ int h3attn_tail_correct(const h3attn_plan* plan, const uint16_t* v, const int32_
                         void* ws, size_t ws_bytes, void* tail_ws, size_t tail_ws_bytes, void* stream) {
   if (!plan_ok(plan) || plan->n_video_blocks == 0) return H3ATTN_EINVAL;
   if (v == nullptr || kv_sel == nullptr || o == nullptr || lse == nullptr) return H3ATTN_EINVAL;
-  const WsLayout w = ws_layout(plan->H, plan->d, plan->n_blocks, plan->n_video_blocks);
+  const WsLayout w = ws_layout(plan);
   if (ws == nullptr || ws_bytes < w.total) return H3ATTN_EWORKSPACE;
   if (tail_ws == nullptr || tail_ws_bytes < h3attn_tail_workspace_bytes(plan)) return H3ATTN_EWORKSPACE;
   if (!aligned16(v) || !aligned16(o) || !aligned16(tail_ws) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||

@@ -291,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   // Tile order: head-major, so the ~300 CTAs resident at a time share one or
   // two heads' K/V in L2; inside a head the dense (prefix) query tiles come
   // first, so the longest tiles start earliest.
-  const int n_qtiles = (p.n_blocks + 1) >> 1;
+  const int n_qtiles = p.n_dense_tiles + p.n_paired_tiles;
   const int head = (int)(blockIdx.x / n_qtiles);
   const int qtile = (int)(blockIdx.x % n_qtiles);
   // An earlier CTA that gave up leaves the status word set: skip the work
@@ -326,9 +326,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     tmem_relinquish();
   }
 
+  // ---- the tile's two query blocks: adjacent ones over the dense prefix,
+  // else the pair chosen by routed-list overlap (qb_b = -1: block a alone)
+  int qb_a = 2 * qtile, qb_b = 2 * qtile + 1;
+  if (qtile >= p.n_dense_tiles) {
+    const uint32_t e = __ldg(p.qpairs + (size_t)head * p.n_paired_tiles + (qtile - p.n_dense_tiles));
+    qb_a = (int)(e & 0xFFFFu);
+    qb_b = (e >> 16) == kNoPair ? -1 : (int)(e >> 16);
+  }
+  const bool has_a = qb_a < p.n_blocks, has_b = qb_b >= 0 && qb_b < p.n_blocks;
+
   // ---- key-block list of this tile: union of the two query blocks' lists ----
-  const int qb_a = 2 * qtile, qb_b = 2 * qtile + 1;
-  const bool has_a = qb_a < p.n_blocks, has_b = qb_b < p.n_blocks;
   const bool dense_a = p.kv_sel == nullptr || qb_a < p.first_video_block;
   const bool dense_b = p.kv_sel == nullptr || qb_b < p.first_video_block;
   for (int w = tid; w < nwords; w += kThreads) {
@@ -403,17 +411,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (warp == 0 && lane == 0) {
       // ---------------------------------------------------------- producer
       uint32_t issued_k = 0, issued_v = 0;
-      const int q_row0 = qtile * kTileRows;
+      const int oob_row = p.n_blocks * 64;  // a whole block past S: zero-filled by TMA
+      const int qa_row = has_a ? qb_a * 64 : oob_row, qb_row = has_b ? qb_b * 64 : oob_row;
       uint8_t* sq = smem + L::kQ;
       uint8_t* sk = smem + L::kK;
       uint8_t* sv = smem + L::kV;
       mbar_arrive_expect_tx(bars.q_full, L::kTileBytes);
 #pragma unroll
       for (int c = 0; c < L::kHalves; ++c) {
-        tma_load_3d(sq + c * L::kHalfBytes, &tm_q, bars.q_full, c * 64, q_row0, head);
-        tma_load_3d(sq + c * L::kHalfBytes + 8192, &tm_q, bars.q_full, c * 64, q_row0 + 64, head);
+        tma_load_3d(sq + c * L::kHalfBytes, &tm_q, bars.q_full, c * 64, qa_row, head);
+        tma_load_3d(sq + c * L::kHalfBytes + 8192, &tm_q, bars.q_full, c * 64, qb_row, head);
       }
-      const int oob_row = p.n_blocks * 64;  // a whole block past S: zero-filled by TMA
       for (int j = 0; j < n_tiles; ++j) {
         const uint32_t ph = (uint32_t)j & 1u;
         const int r0 = (int)(list[2 * j] & 0x3FFFu) * 64;
@@ -530,8 +538,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint8_t* ph1_row = smem + L::kPh1 + part * L::kPh1StepBytes + r * 32;
     const uint32_t ph1_swz = (uint32_t)((r >> 2) & 1) << 4;  // 32-byte swizzle: bit 4 ^= bit 7
     const int my_bit = 14 + (r >> 6);  // list bit of this row's query block
-    const int qrow = qtile * kTileRows + r;
-    const bool row_valid = qrow < p.S;
+    const int qrow = (r < 64 ? qb_a : qb_b) * 64 + (r & 63);
+    const bool row_valid = (r < 64 ? has_a : has_b) && qrow < p.S;
     const bool pen_row = p.pen_on && row_valid && p.seg[qrow] == kSegOutput;
     const float tq = pen_row ? p.times[qrow] : 0.0f;
     const float scale = p.scale_log2;

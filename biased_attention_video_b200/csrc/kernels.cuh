@@ -24,6 +24,10 @@ struct AttnParams {
   const uint4* kv_desc;        // [n_blocks]: see launch_kv_desc
   const float* gtime;          // [n_blocks * 64]: guide key's time, NaN for other keys (read for kind 2)
   const uint32_t* slow_blocks; // [ceil(n_blocks / 32)] bitmap: blocks needing per-key treatment
+  // tiles per head: n_dense_tiles of adjacent blocks (2t, 2t+1), then
+  // n_paired_tiles read from qpairs[H][n_paired_tiles] (see launch_pair)
+  const uint32_t* qpairs;
+  int n_dense_tiles, n_paired_tiles;
   uint16_t* o;                 // bf16 [H][S][d]
   float* lse;                  // [H][S] or null
   int* status;                 // device status word
@@ -51,6 +55,23 @@ cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUte
 // 16-key group), for every block b < 32 ceil(n_blocks / 32).
 cudaError_t launch_kv_desc(const uint8_t* seg, const float* times, int S, int n_blocks, uint4* kv_desc,
                            float* gtime, uint32_t* slow, cudaStream_t stream);
+
+// Query-block pairing (pair.cu).  With routing, the attention tiles of a head
+// are the adjacent pairs (2t, 2t+1) of blocks below paired_first_block(fvb)
+// (the dense prefix, rounded up to an even block), then paired_tiles(...)
+// tiles of blocks from that point on, paired within groups of kPairGroup
+// consecutive blocks by routed-list overlap.  Entry: block a | block b << 16,
+// b = kNoPair for a tile holding block a alone.
+constexpr int kPairGroup = 32;
+constexpr uint32_t kNoPair = 0xFFFFu;
+inline int paired_first_block(int first_video_block) { return (first_video_block + 1) & ~1; }
+inline int paired_tiles(int n_blocks, int first_video_block) {
+  const int n = n_blocks - paired_first_block(first_video_block);
+  return n <= 0 ? 0 : n / kPairGroup * (kPairGroup / 2) + (n % kPairGroup + 1) / 2;
+}
+// pairs[H][paired_tiles(n_blocks, first_video_block)] from kv_sel[H][nV][k]
+cudaError_t launch_pair(const int32_t* kv_sel, int H, int n_blocks, int first_video_block, int k,
+                        uint32_t* pairs, cudaStream_t stream);
 
 // mean-pool blocks [first_block, first_block + n_out) of up to two bf16 [H][S][d] tensors
 cudaError_t launch_pool(const uint16_t* x0, float* out0, const uint16_t* x1, float* out1, int H, int S,

@@ -117,7 +117,9 @@ H3ATTN_API int h3attn_plan_init(h3attn_plan* plan, int H, int S, int d, int bloc
 /* Bytes of device workspace a plan needs for h3attn_route and h3attn_forward
  * (status word; the attention scratch: per-block key descriptors, per-key
  * guide times and a bitmap of the key blocks that need per-key handling,
- * about 0.5 MB at S = 116,883; and the routing scratch: two-part bf16 pooled
+ * about 0.5 MB at S = 116,883; the query-block pair table of a routed
+ * forward, 4 bytes per head and 128-row tile of video query blocks, about
+ * 0.2 MB at S = 116,883, H = 56; and the routing scratch: two-part bf16 pooled
  * Q and K of the video blocks and the fp32 pooled-score matrix, about 0.9 GB
  * at S = 116,883, H = 56, d = 128).
  * The caller allocates it once, zero-filled (the first 256 bytes hold the
@@ -171,7 +173,13 @@ H3ATTN_API int h3attn_route_static(const h3attn_plan* plan, const uint16_t* q, c
  * o: bf16 [H][S][d] device (rounded to nearest even); lse: float32 [H][S]
  * device natural-log normaliser, or NULL.
  * Routed indices outside [first_video_block, n_blocks) are ignored and flagged
- * (H3ATTN_EDATA from h3attn_check). */
+ * (H3ATTN_EDATA from h3attn_check).
+ * ws: the workspace (h3attn_workspace_bytes(plan) bytes always suffices); a
+ * call with kv_sel NULL reads and writes only its status word and attention
+ * scratch, a routed call also the pair table that follows them.  The routed
+ * call pairs its video query blocks into 128-row tiles by the overlap of their
+ * routed lists (groups of 32 consecutive blocks, greedy largest overlap first);
+ * the pairing affects only the speed, not which keys a row attends. */
 H3ATTN_API int h3attn_forward(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                    const uint8_t* seg, const float* times, const h3attn_penalty* pen,
                    const int32_t* kv_sel, uint16_t* o, float* lse, void* ws, size_t ws_bytes,

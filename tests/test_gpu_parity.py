@@ -130,6 +130,17 @@ def test_forward_routed_ragged(d, segs, sparsity):
     _forward_all_rows(cfg, sparsity, PEN, routed=True)
 
 
+@pytest.mark.parametrize("sparsity", [0.5, 0.9])
+def test_forward_routed_paired_groups(sparsity):
+    """Odd first video block (3): the dense prefix ends on a mixed tile (2, 3)
+    and the overlap pairing covers blocks 4..100, three full groups of 32 and
+    one lone block; every row of both heads checked."""
+    segs = _layout(100, 30, 3, 300, 9, 600)
+    cfg = inputs.custom(2, 128, segs, seed=55, cluster_norm=2.0)
+    _, p = _forward_all_rows(cfg, sparsity, PEN, routed=True)
+    assert p.first_video_block == 3 and p.n_blocks == 101
+
+
 def test_config1_dense_biased():
     cfg = inputs.CONFIGS[1]
     x = make(cfg)
