@@ -78,8 +78,8 @@ struct Layout {
   static constexpr int kPh1 = kV + kTileBytes;
   static constexpr int kPh1StepBytes = kTileRows * 32;
   static constexpr int kBars = kPh1 + 2 * kPh1StepBytes;
-  // q_full, k_full, k_empty, v_full, v_empty, s_full, p_full[2], o_half0, o_done, o_final, drain, xchg[4]
-  static constexpr int kNumBars = 16;
+  // q_full, k_full, k_empty, v_full, v_empty, s_full, p_full[2], o_done, o_final, drain, xchg[4]
+  static constexpr int kNumBars = 15;
   static constexpr int kMisc = kBars + kNumBars * 8;  // tmem base, abort flag, n_entries, n_fast
   static constexpr int kRed = kMisc + 16;             // partial row maxima / sums: float [2][2][128]
   static constexpr int kBitmaps = kRed + 2 * 2 * 128 * 4;
@@ -90,21 +90,21 @@ struct Layout {
 };
 
 struct Bars {
-  uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *o_half0, *o_done, *o_final, *drain,
-      *xchg;
+  uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *s_full, *p_full, *o_done, *o_final, *drain, *xchg;
 };
 
 // p_full[ph]: P of phase ph of the current tile is in place (one completion
 // per tile each, so a waiter is never more than one phase behind).
-// o_half0 / o_done: PV(j, phase 0) / PV(j, phase 1) complete.  The softmax
-// waits for both on every tile (o_done(j-1) in phase 0 of tile j, o_half0(j)
-// in phase 1), so its parity never falls behind either.
+// o_done: PV(j, phase 1) complete, hence all of tile j's MMAs (one thread
+// issues them, and they run in issue order).  The softmax waits for it on
+// every tile (o_done(j-1) in phase 0 of tile j), so its parity never falls
+// behind.
 // xchg[q]: the two softmax warps of TMEM lane quarter q have written their
 // partial row values (64 arrivals per exchange; neither warp can run more than
 // one exchange ahead of the other).
 __device__ __forceinline__ Bars carve_bars(uint8_t* base) {
   uint64_t* b = reinterpret_cast<uint64_t*>(base);
-  return Bars{b, b + 1, b + 2, b + 3, b + 4, b + 5, b + 6, b + 8, b + 9, b + 10, b + 11, b + 12};
+  return Bars{b, b + 1, b + 2, b + 3, b + 4, b + 5, b + 6, b + 8, b + 9, b + 10, b + 11};
 }
 
 // Bounded wait with CTA-wide abort.  On give-up: raise the CTA abort flag and
@@ -311,7 +311,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     mbar_init(bars.s_full, 1);
     mbar_init(bars.p_full, 8);
     mbar_init(bars.p_full + 1, 8);
-    mbar_init(bars.o_half0, 1);
     mbar_init(bars.o_done, 1);
     mbar_init(bars.o_final, 1);
     mbar_init(bars.drain, 1);
@@ -489,7 +488,6 @@ __global__ void __launch_bounds__(kThreads, 2)
             const uint64_t bdesc = sw128_desc(v_addr + (4 * b + c) * 2048, L::kHalfBytes, 1024);
             umma_ts(tmem_o, tmem_s + 64 * b + 8 * c, bdesc, kIdescO, (j > 0 || b > 0 || c > 0) ? 1u : 0u);
           }
-        umma_commit(bars.o_half0);
         // S(j+1): every thread has read its phase-1 scores before p_full[0]
         if (j + 1 < n_tiles && !issue_s(j + 1)) {
           ok = false;
@@ -547,9 +545,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     float l = 0.0f;       // partial row sum over this thread's keys
     bool ok = true;
 
-    // Combine this thread's partial max with its partner's (slot `slot`: a
-    // slot is rewritten only after the next exchange's barrier, which both
-    // threads pass after reading it).  Returns false on give-up.
+    // Combine this thread's partial max with its partner's.  Exchanges
+    // alternate between two slots: a thread writes slot s again only after
+    // passing the next exchange's barrier, which its partner reaches only
+    // after reading slot s.  Returns false on give-up.
     auto exchange_max = [&](float pmax, int slot, float& mx) -> bool {
       red[(slot * 2 + part) * 128 + r] = pmax;
       mbar_arrive(xbar);
@@ -604,29 +603,36 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       tc_fence_after();
 
-      // ---------------- phase 0: keys 0..47 of the block, P back into TMEM
-      float sv[kPhase0Keys];
+      // All 64 scores of this thread's block: one max and one partner
+      // exchange per tile, for both phases (the phase-1 scores are read
+      // again after phase 0, to keep them out of phase 0's registers).
+      float sv[kPhase0Keys], sv1[16];
       {
-        uint32_t t32[32], t16[16];
+        uint32_t t32[32], t16[16], u16[16];
         __syncwarp();
         tmem_ld32(t_s, t32);
         tmem_ld16(t_s + 32, t16);
+        tmem_ld16(t_s + kPhase0Keys, u16);
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i) sv[i] = __uint_as_float(t32[i]);
 #pragma unroll
         for (int i = 0; i < 16; ++i) sv[32 + i] = __uint_as_float(t16[i]);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sv1[i] = __uint_as_float(u16[i]);
       }
       float mx;
-      if (!exchange_max(kGeneral ? part_max<kPhase0Keys>(sv, bm, 0) : full_max<kPhase0Keys>(sv, bm), 0, mx)) {
-        return false;
-      }
+      const float pmax = kGeneral ? fmaxf(part_max<kPhase0Keys>(sv, bm, 0), part_max<16>(sv1, bm, kPhase0Keys))
+                                  : fmaxf(full_max<kPhase0Keys>(sv, bm), full_max<16>(sv1, bm));
+      if (!exchange_max(pmax, j & 1, mx)) return false;
       // Conditional rescale: the running max only moves when it grows by more
       // than 2^8; below that the stale max keeps every probability <= 256.
-      bool grow = mx > m + kRescaleThreshold;
-      bool o_rescale = grow && m > -INFINITY;
-      float m_old = m;
+      const bool grow = mx > m + kRescaleThreshold;
+      const bool o_rescale = grow && m > -INFINITY;
+      const float m_old = m;
       if (grow) m = mx;
+
+      // ---------------- phase 0: keys 0..47 of the block, P back into TMEM
       float lt = 0.0f;
 #pragma unroll
       for (int g = 0; g < kPhase0Keys / 16; ++g) {
@@ -636,9 +642,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         __syncwarp();
         tmem_st8(t_s + 8 * g, pk);  // P of keys 16g..16g+15 over score columns 8g..8g+7
       }
-      // phase-1 scores: read now, so that S(j+1) may overwrite the S region
-      // as soon as PV(j, phase 0) has consumed P
-      float sv1[16];
+      // phase-1 scores again: S(j+1) may overwrite the S region as soon as
+      // PV(j, phase 0) has consumed P, which follows p_full[0]
       {
         uint32_t t16[16];
         __syncwarp();
@@ -665,14 +670,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.p_full);  // one arrival per softmax warp
 
-      // ---------------- phase 1: keys 48..63, P to shared memory
-      if (!exchange_max(kGeneral ? part_max<16>(sv1, bm, kPhase0Keys) : full_max<16>(sv1, bm), 1, mx)) {
-        return false;
-      }
-      grow = mx > m + kRescaleThreshold;
-      o_rescale = grow && m > -INFINITY;
-      m_old = m;
-      if (grow) m = mx;
+      // ---------------- phase 1: keys 48..63 (same max), P to shared memory
       {
         // PV(j-1, phase 1) read the previous contents: complete (o_done above)
         uint32_t pk[8];
@@ -682,17 +680,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         *reinterpret_cast<uint4*>(ph1_row + (16u ^ ph1_swz)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
       }
       fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor core
-      alpha = 1.0f;
-      if (!__all_sync(kFull, wait_bar(bars.o_half0, ph, p, abort_flag))) {
-        return false;
-      }
-      tc_fence_after();
-      if (__any_sync(kFull, o_rescale)) {
-        alpha = o_rescale ? ex2(m_old - m) : 1.0f;
-        rescale_o(alpha);
-        tmem_wait_st();
-      }
-      l = l * alpha + lt;
+      l += lt;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.p_full + 1);
@@ -703,13 +691,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (; ok && j < n_tiles; ++j) ok = tile(j, std::true_type{});
     // ---------------------------------------------------------- epilogue
     bool fin = __all_sync(kFull, ok) && n_tiles > 0;
-    // total row sum: slot 0 is free here (its last reader passed the barrier
-    // of the final phase-1 exchange before this thread did)
+    // total row sum, in the slot the last tile's exchange did not use
     if (fin) {
-      red[part * 128 + r] = l;
+      const int slot = n_xchg & 1u;
+      red[(slot * 2 + part) * 128 + r] = l;
       mbar_arrive(xbar);
       fin = wait_bar(xbar, n_xchg & 1u, p, abort_flag);
-      if (fin) l += red[(part ^ 1) * 128 + r];
+      if (fin) l += red[(slot * 2 + (part ^ 1)) * 128 + r];
       if (fin) fin = wait_bar(bars.o_final, 0, p, abort_flag);
     }
     if (__all_sync(kFull, fin)) {
