@@ -572,6 +572,44 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     };
 
+    // The tile for a warp whose rows do not attend this thread's key block.
+    auto skip_tile = [&](int j) -> bool {
+      const uint32_t ph = (uint32_t)j & 1u;
+      const uint32_t zero[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int g = 0; g < kPhase0Keys / 16; ++g) {
+        __syncwarp();
+        tmem_st8(t_s + 8 * g, zero);
+      }
+      float mx;
+      if (!exchange_max(-INFINITY, j & 1, mx)) return false;
+      const bool grow = mx > m + kRescaleThreshold;
+      const bool o_rescale = grow && m > -INFINITY;
+      const float m_old = m;
+      if (grow) m = mx;
+      if (j > 0) {
+        if (!__all_sync(kFull, wait_bar(bars.o_done, ph ^ 1u, p, abort_flag))) return false;
+        tc_fence_after();
+      }
+      float alpha = 1.0f;
+      if (__any_sync(kFull, o_rescale)) {
+        alpha = o_rescale ? ex2(m_old - m) : 1.0f;
+        rescale_o(alpha);
+      }
+      l *= alpha;
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.p_full);
+      *reinterpret_cast<uint4*>(ph1_row) = make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(ph1_row + 16) = make_uint4(0u, 0u, 0u, 0u);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.p_full + 1);
+      return true;
+    };
+
     // One tile; kGeneral selects the per-key path (validity, per-key penalty)
     // that the few slow key blocks need -- kept out of the loop over the
     // others so that it does not weigh on their register allocation.
@@ -602,6 +640,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         return false;
       }
       tc_fence_after();
+      // A warp's 32 rows belong to one query block: when that block does not
+      // attend this key block (the tile's other block does), the warp writes
+      // zero probabilities without reading the scores; it still takes part in
+      // the exchange and in any rescale of its rows.
+      if (__all_sync(kFull, !attended)) return skip_tile(j);
 
       // All 64 scores of this thread's block: one max and one partner
       // exchange per tile, for both phases (the phase-1 scores are read
