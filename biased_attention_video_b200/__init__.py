@@ -38,7 +38,7 @@ class H3Error(RuntimeError):
 
 class Plan(ctypes.Structure):
     _fields_ = [("H", ctypes.c_int32), ("S", ctypes.c_int32), ("d", ctypes.c_int32), ("block", ctypes.c_int32),
-                ("sparsity", ctypes.c_float), ("n_blocks", ctypes.c_int32), ("prefix_rows", ctypes.c_int32),
+                ("sparsity", ctypes.c_double), ("n_blocks", ctypes.c_int32), ("prefix_rows", ctypes.c_int32),
                 ("first_video_block", ctypes.c_int32), ("n_forced", ctypes.c_int32),
                 ("n_video_blocks", ctypes.c_int32), ("k", ctypes.c_int32)]
 
@@ -68,7 +68,7 @@ def lib():
         path = _build.build()
         L = ctypes.CDLL(path)
         PP = ctypes.POINTER(Plan)
-        L.h3attn_plan_init.argtypes = [PP, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, _P]
+        L.h3attn_plan_init.argtypes = [PP, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, _P]
         L.h3attn_plan_init.restype = ctypes.c_int
         L.h3attn_workspace_bytes.argtypes = [PP]
         L.h3attn_workspace_bytes.restype = ctypes.c_size_t

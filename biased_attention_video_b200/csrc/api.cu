@@ -179,9 +179,9 @@ bool encode_bf16_3d(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t 
 
 extern "C" {
 
-int h3attn_plan_init(h3attn_plan* plan, int H, int S, int d, int block, float sparsity, const uint8_t* seg_host) {
+int h3attn_plan_init(h3attn_plan* plan, int H, int S, int d, int block, double sparsity, const uint8_t* seg_host) {
   if (plan == nullptr || seg_host == nullptr || H <= 0 || S <= 0) return H3ATTN_EINVAL;
-  if (!(sparsity >= 0.0f && sparsity < 1.0f)) return H3ATTN_EINVAL;
+  if (!(sparsity >= 0.0 && sparsity < 1.0)) return H3ATTN_EINVAL;
   if (!(d == 64 || d == 128) || block != h3::kBlock) return H3ATTN_EUNSUPPORTED;
   const int n_blocks = (S + block - 1) / block;
   if (n_blocks > h3::kMaxBlocks) return H3ATTN_EUNSUPPORTED;
@@ -203,7 +203,7 @@ int h3attn_plan_init(h3attn_plan* plan, int H, int S, int d, int block, float sp
   p.n_forced = p.first_video_block;
   p.n_video_blocks = n_blocks - p.first_video_block;
   if (p.n_video_blocks > 0) {
-    const double want = std::ceil((1.0 - (double)sparsity) * (double)p.n_video_blocks - 1e-9);
+    const double want = std::ceil((1.0 - sparsity) * (double)p.n_video_blocks - 1e-9);
     int kk = (int)want;
     if (kk < 1) kk = 1;
     if (kk > p.n_video_blocks) kk = p.n_video_blocks;
@@ -410,7 +410,7 @@ int h3attn_dense_biased(int H, int S, int d, const uint16_t* q, const uint16_t* 
   p.S = S;
   p.d = d;
   p.block = h3::kBlock;
-  p.sparsity = 0.0f;
+  p.sparsity = 0.0;
   p.n_blocks = (S + h3::kBlock - 1) / h3::kBlock;
   if (p.n_blocks > h3::kMaxBlocks) return H3ATTN_EUNSUPPORTED;
   p.prefix_rows = S;

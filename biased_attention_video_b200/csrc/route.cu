@@ -355,6 +355,122 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ sco
   }
 }
 
+// Register-resident top-k for rows of at most 32 NPL scores (one warp per
+// (head, video query block)); the same selection as topk_kernel: the k
+// highest scores, ties to the lower block, listed in ascending block order.
+// Lane l holds the scores j = l + 32 i (i < NPL) as order-preserving integer
+// keys (-0 folded into +0 first, so equal floats give equal keys; padding
+// past n_video gets key 0, below every real key).  The candidates are always
+// a contiguous key range [alo, ahi]: each level bins that range into 256
+// bins of 2^shift keys, takes every key above the bin that holds the next
+// needed key, and narrows the range to that bin.  shift drops by 8 per
+// level, so after at most four levels the range is one key and its keys go
+// by ascending block; shared memory holds only the warp's histogram.
+template <int NPL>
+__global__ void __launch_bounds__(256, 2) topk_reg_kernel(const float* __restrict__ scores, int32_t* __restrict__ sel,
+                                                          int rows, int n_video, int ldc, int k, int first_video_block) {
+  __shared__ uint32_t hist_all[8][256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + warp;
+  if (row >= rows) return;  // warp-uniform
+  uint32_t* hist = hist_all[warp];
+  const unsigned full = 0xFFFFFFFFu;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  const float* src = scores + (size_t)row * ldc;
+
+  uint32_t key[NPL];
+  uint32_t alo = 0xFFFFFFFFu, ahi = 0u;
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    const int j = lane + 32 * i;
+    key[i] = 0u;
+    if (j < n_video) {
+      const uint32_t b = __float_as_uint(__ldg(src + j) + 0.0f);
+      key[i] = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+      alo = min(alo, key[i]);
+      ahi = max(ahi, key[i]);
+    }
+  }
+  alo = __reduce_min_sync(full, alo);
+  ahi = __reduce_max_sync(full, ahi);
+  int need = k;
+  bool ties = false;  // finished with every key of [alo, ahi] equal: take `need` of them by block
+  for (int level = 0; level < 5; ++level) {
+    if (alo == ahi) {
+      ties = true;
+      break;
+    }
+    const uint32_t span = ahi - alo;
+    const int shift = span < 256u ? 0 : (32 - __clz((int)span)) - 8;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) hist[lane * 8 + e] = 0u;
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < NPL; ++i)
+      if (key[i] >= alo && key[i] <= ahi) atomicAdd(hist + ((key[i] - alo) >> shift), 1u);
+    __syncwarp();
+    // bin T holding the need-th best: lane l owns bins 255-8l .. 248-8l (descending)
+    uint32_t c[8], sum = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      c[e] = hist[255 - 8 * lane - e];
+      sum += c[e];
+    }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(full, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const uint32_t excl = incl - sum;
+    const bool here = excl < (uint32_t)need && (uint32_t)need <= incl;
+    const int src_lane = __ffs((int)__ballot_sync(full, here)) - 1;
+    uint32_t tbin = 0, greater = 0, in_bin = 0, cum = excl;
+    bool found = false;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      if (here && !found && cum + c[e] >= (uint32_t)need) {
+        found = true;
+        tbin = 255 - 8 * lane - e;
+        greater = cum;
+        in_bin = c[e];
+      }
+      cum += c[e];
+    }
+    tbin = __shfl_sync(full, tbin, src_lane);
+    greater = __shfl_sync(full, greater, src_lane);
+    in_bin = __shfl_sync(full, in_bin, src_lane);
+    __syncwarp();  // every lane has read the histogram before the next level clears it
+    // keys above bin T are taken; the candidates narrow to bin T
+    // (bin T holds a key, so blo <= ahi; no sum below can wrap)
+    const uint32_t blo = alo + (tbin << shift);
+    ahi = blo + min((1u << shift) - 1u, ahi - blo);
+    alo = blo;
+    need -= (int)greater;
+    if ((uint32_t)need == in_bin) break;  // the whole bin is taken: keys >= alo
+  }
+  // selected: keys above the range, and, when the range is one tied key,
+  // its `need` lowest blocks; else (the whole last bin) every key >= alo
+  int32_t* dst = sel + (size_t)row * k;
+  int pos = 0, tie_seen = 0;
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    bool t;
+    if (ties) {
+      const bool tie = key[i] == alo;
+      const uint32_t tm = __ballot_sync(full, tie);
+      t = key[i] > alo || (tie && tie_seen + __popc(tm & lt_mask) < need);
+      tie_seen += __popc(tm);
+    } else {
+      t = key[i] >= alo;
+    }
+    const uint32_t m = __ballot_sync(full, t);
+    const int slot = pos + __popc(m & lt_mask);
+    if (t && slot < k) dst[slot] = first_video_block + lane + 32 * i;
+    pos += __popc(m);
+  }
+}
+
 }  // namespace
 
 RouteScratch route_scratch_layout(int H, int d, int n_video) {
@@ -400,14 +516,28 @@ cudaError_t launch_route_pipeline(const uint16_t* q, const uint16_t* k, int32_t*
   score_gemm_kernel<<<ggrid, kGemmThreads, kGSmem, stream>>>(ta, tb, sc, n_video, (int)r.ldc, 3 * d / 64, status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  // 3. top-k per (head, query block)
+  // 3. top-k per (head, query block): scores in registers up to 2048 video
+  // blocks, else staged in shared memory
+  const int rows = H * n_video;
+  const unsigned rgrid = (unsigned)((rows + 7) / 8);
+  if (n_video <= 2048) {
+    const int npl = (n_video + 31) / 32;
+    if (npl <= 16)
+      topk_reg_kernel<16><<<rgrid, 256, 0, stream>>>(sc, kv_sel, rows, n_video, (int)r.ldc, kk, first_video_block);
+    else if (npl <= 32)
+      topk_reg_kernel<32><<<rgrid, 256, 0, stream>>>(sc, kv_sel, rows, n_video, (int)r.ldc, kk, first_video_block);
+    else if (npl <= 48)
+      topk_reg_kernel<48><<<rgrid, 256, 0, stream>>>(sc, kv_sel, rows, n_video, (int)r.ldc, kk, first_video_block);
+    else
+      topk_reg_kernel<64><<<rgrid, 256, 0, stream>>>(sc, kv_sel, rows, n_video, (int)r.ldc, kk, first_video_block);
+    return cudaGetLastError();
+  }
   const int words = topk_warp_words(n_video, (int)r.ldc);
   int wpc = (int)((200 * 1024) / (words * 4));
   wpc = wpc < 1 ? 1 : (wpc > 8 ? 8 : wpc);
   const size_t tsmem = (size_t)wpc * words * 4;
   e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsmem);
   if (e != cudaSuccess) return e;
-  const int rows = H * n_video;
   topk_kernel<<<(rows + wpc - 1) / wpc, wpc * 32, tsmem, stream>>>(sc, kv_sel, rows, n_video, (int)r.ldc, kk,
                                                                    first_video_block);
   return cudaGetLastError();

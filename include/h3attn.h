@@ -100,10 +100,12 @@ typedef struct {
  *  n_forced          = first_video_block: key blocks always attended, and
  *                    query blocks attended densely (they hold a non-video row)
  *  n_video_blocks    n_blocks - first_video_block (nV)
- *  k                 routed video key blocks per video query block */
+ *  k                 routed video key blocks per video query block:
+ *                    ceil((1 - sparsity) nV), at least 1 (a product within
+ *                    1e-9 above an integer counts as that integer) */
 typedef struct {
   int32_t H, S, d, block;
-  float sparsity;
+  double sparsity;
   int32_t n_blocks, prefix_rows, first_video_block, n_forced, n_video_blocks, k;
 } h3attn_plan;
 
@@ -111,7 +113,7 @@ typedef struct {
  * 0 <= sparsity < 1; rows with seg 3/4 (video) must form a contiguous suffix
  * of the sequence ("Flash Partitions ...", section 7: contiguous video rows).
  * A sequence without video rows is accepted (no routing; everything dense). */
-H3ATTN_API int h3attn_plan_init(h3attn_plan* plan, int H, int S, int d, int block, float sparsity,
+H3ATTN_API int h3attn_plan_init(h3attn_plan* plan, int H, int S, int d, int block, double sparsity,
                      const uint8_t* seg_host);
 
 /* Bytes of device workspace a plan needs for h3attn_route and h3attn_forward

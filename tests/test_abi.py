@@ -136,3 +136,16 @@ def test_host_validation_before_any_device_work():
     assert L.h3attn_workspace_bytes(ctypes.byref(p)) == 0
     for code in [0, -1, -2, -3, -4, -5, -6, -7, -99]:
         assert isinstance(L.h3attn_strerror(code), bytes)
+
+
+def test_plan_k_matches_oracle_for_decimal_sparsities():
+    """k = ceil((1 - sparsity) nV) read in double precision: 0.9 of 2,100 video
+    blocks keeps 210 (a float 0.9 would give 211)."""
+    import oracle
+    for nv, sp in [(2100, 0.9), (1794, 0.9), (100, 0.85), (7, 0.5), (8000, 0.95), (3, 0.0)]:
+        S = 64 + nv * 64
+        seg = np.array([0] * 64 + [4] * (nv * 64), np.uint8)
+        p = h3.plan(1, S, 64, seg, sparsity=sp)
+        assert p.n_video_blocks == nv
+        assert p.k == oracle.k_for(nv, sp), (nv, sp, p.k)
+    assert h3.plan(1, 64 + 2100 * 64, 64, np.array([0] * 64 + [4] * 2100 * 64, np.uint8), sparsity=0.9).k == 210

@@ -68,6 +68,31 @@ def test_route_config3_sampled_heads(sparsity):
     _route_and_compare(inputs.CONFIGS[3], sparsity, heads=[0, 27, 55])
 
 
+def test_route_more_than_2048_video_blocks():
+    """2,100 video blocks: past the register-resident top-k (2,048), so the
+    shared-memory one selects; one head, d = 64."""
+    segs = _layout(64, 0, 0, 0, 30, 70 * 64)
+    cfg = inputs.custom(1, 64, segs, seed=17, cluster_norm=2.0)
+    p, _, _, _ = _route_and_compare(cfg, 0.9)
+    assert p.n_video_blocks == 2100
+
+
+def test_route_many_equal_scores():
+    """Repeated key blocks make whole groups of equal pooled scores: the
+    selection must still take the lowest blocks of a tied group."""
+    segs = _layout(64, 0, 0, 0, 12, 64 * 20)
+    cfg = inputs.custom(2, 128, segs, seed=23, cluster_norm=2.0)
+    x = make(cfg, device=None)
+    k = x["k"].copy()
+    for b in range(1, cfg.S // 64):
+        k[:, b * 64:(b + 1) * 64] = k[:, (1 + b % 7) * 64:(2 + b % 7) * 64]   # 7 distinct video key blocks
+    p = h3.plan(2, cfg.S, 128, x["seg"], sparsity=0.7)
+    ws = h3.workspace(p)
+    sel = h3.route(p, dev_bf16(x["q"]), dev_bf16(k), ws).cpu().numpy()
+    ref, _, _ = oracle.route(x["q"], k, x["seg"], 0.7)
+    assert np.array_equal(sel, ref)
+
+
 def test_route_tie_goes_to_lower_block():
     segs = _layout(64, 0, 0, 0, 8, 64)
     cfg = inputs.custom(2, 128, segs, seed=5, cluster_norm=2.0)
