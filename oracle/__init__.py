@@ -62,6 +62,11 @@ def lib():
         L.oracle_tail.argtypes = [ctypes.c_int] * 4 + [_P] * 5 + [ctypes.c_int, _P, _P]
         L.oracle_tail.restype = None
         L.oracle_threads.restype = ctypes.c_int
+        L.oracle_quantize_rows.argtypes = [ctypes.c_long, ctypes.c_int, _P, _P, _P]
+        L.oracle_quantize_rows.restype = None
+        L.oracle_attend_qk8.argtypes = [ctypes.c_int] * 4 + [_P, _P, _P, _P, ctypes.c_int] + [_P] * 5 + \
+            [ctypes.c_int, _P, _P, _P, _P]
+        L.oracle_attend_qk8.restype = None
         _lib = L
     return _lib
 
@@ -162,6 +167,45 @@ def attend(q, k, v, seg, times, pen=None, sel=None, heads=None, rows=None, B: in
         heads = np.repeat(np.arange(H), S)
         rows = np.tile(np.arange(S), H)
     return _attend(lib().oracle_attend, q, k, v, seg, times, pen, sel, heads, rows, B)
+
+
+def quantize_rows(x):
+    """Per-token int8 quantisation ("H3 SLA Attention", inputs table, use_int8_qk) of bf16 bit patterns
+    x [..., d]: per row s = max|x| / 127 and codes rint(x * (127 / max|x|)) clamped to +-127, in fp32 with
+    ties to even; a zero row gets s = 0.  Returns (codes int8 [..., d], scales float32 [...])."""
+    x = _c(x, np.uint16)
+    d = x.shape[-1]
+    n = x.size // d
+    codes = np.empty(x.shape, np.int8)
+    scales = np.empty(x.shape[:-1], np.float32)
+    lib().oracle_quantize_rows(n, d, x.ctypes.data, codes.ctypes.data, scales.ctypes.data)
+    return codes, scales
+
+
+def attend_qk8(q, k, v, seg, times, pen=None, sel=None, heads=None, rows=None, B: int = 64):
+    """As attend, with Q and K quantised per token to int8 before the QK dot product (quantize_rows); the
+    score is s_q s_k (integer dot of the codes) / sqrt(d); PV uses v as given."""
+    q8, sq = quantize_rows(q)
+    k8, sk = quantize_rows(k)
+    v = _c(v, np.uint16)
+    seg = _c(seg, np.uint8)
+    times = _c(times, np.float32)
+    H, S, d = v.shape
+    if rows is None:
+        heads = np.repeat(np.arange(H), S)
+        rows = np.tile(np.arange(S), H)
+    heads = _c(heads, np.int32)
+    rows = _c(rows, np.int32)
+    n = len(rows)
+    pen_arr = None if pen is None else _c(pen, np.float64)
+    sel_c = None if sel is None else _c(sel, np.int32)
+    kk = 0 if sel is None else sel_c.shape[-1]
+    o = np.empty((n, d), np.float64)
+    lse = np.empty(n, np.float64)
+    lib().oracle_attend_qk8(H, S, d, B, seg.ctypes.data, times.ctypes.data, _ptr(pen_arr), _ptr(sel_c), kk,
+                            q8.ctypes.data, sq.ctypes.data, k8.ctypes.data, sk.ctypes.data, v.ctypes.data, n,
+                            heads.ctypes.data, rows.ctypes.data, o.ctypes.data, lse.ctypes.data)
+    return o, lse
 
 
 def attend_partitions(q, k, v, seg, times, pen=None, sel=None, heads=None, rows=None, B: int = 64):

@@ -35,7 +35,9 @@
  *    it overlaps any non-video row; every other block is a video block;
  *  - dropped blocks leave the softmax (no pooled tail term);
  *  - routing ignores the penalty; the exact penalty applies on the routed
- *    output -> guide pairs.
+ *    output -> guide pairs;
+ *  - int8 QK: per-row scale max|x| / 127 and codes rint(x * (127 / max|x|)),
+ *    in fp32 with ties to even.
  *
  * Segment ids: 0 text, 1 image-ref, 2 audio, 3 guide video, 4 output video.
  * bf16 inputs are passed as their 16-bit patterns and widened exactly.
@@ -228,6 +230,20 @@ static inline double raw_score(const uint16_t *qr, const uint16_t *kr, int d, do
     return dot * inv_sqrt_d;
 }
 
+/* Int8 QK operands of the quantised score (oracle_attend_qk8); NULL for the exact one. */
+typedef struct {
+    const int8_t *q8, *k8;  /* codes [H][S][d] */
+    const float *sq, *sk;   /* scales [H][S] */
+} qk8_operands;
+
+/* the quantised score s_q s_k (sum_c cq_c ck_c) / sqrt(d); the integer sum is exact */
+static inline double qk8_score(const qk8_operands *o, size_t qi, size_t kj, int d, double inv_sqrt_d) {
+    const int8_t *qr = o->q8 + qi * d, *kr = o->k8 + kj * d;
+    long dot = 0;
+    for (int c = 0; c < d; ++c) dot += (long)qr[c] * (long)kr[c];
+    return (double)dot * (double)o->sq[qi] * (double)o->sk[kj] * inv_sqrt_d;
+}
+
 /*
  * Direct definition ([FP §1], [WIKI]).  For each requested (head, row):
  *   x_j = q.k_j / sqrt(d) - p_j over the attended keys j,
@@ -237,10 +253,10 @@ static inline double raw_score(const uint16_t *qr, const uint16_t *kr, int d, do
  * sel/kk: routed lists from a routing call, or NULL for dense attention.
  * out_o: [n][d]; out_lse: [n].
  */
-void oracle_attend(int H, int S, int d, int B, const uint8_t *seg, const float *times,
-                   const double *pen, const int32_t *sel, int kk, const uint16_t *q,
-                   const uint16_t *k, const uint16_t *v, int n, const int32_t *heads,
-                   const int32_t *rows, double *out_o, double *out_lse) {
+static void attend_core(int H, int S, int d, int B, const uint8_t *seg, const float *times,
+                        const double *pen, const int32_t *sel, int kk, const uint16_t *q,
+                        const uint16_t *k, const uint16_t *v, const qk8_operands *qk8, int n,
+                        const int32_t *heads, const int32_t *rows, double *out_o, double *out_lse) {
     int nkb = (S + B - 1) / B;
     uint8_t *nonvideo = (uint8_t *)malloc((size_t)nkb);
     oracle_block_classes(S, B, seg, nonvideo);
@@ -257,12 +273,13 @@ void oracle_attend(int H, int S, int d, int B, const uint8_t *seg, const float *
         for (int t = 0; t < n; ++t) {
             int h = heads[t], i = rows[t];
             attended_blocks(nkb, nonvideo, vid_index, sel, kk, H, nv, h, i / B, use);
-            const uint16_t *qr = q + ((size_t)h * S + i) * d;
+            const uint16_t *qr = q != NULL ? q + ((size_t)h * S + i) * d : NULL;
             int biased_row = pen != NULL && seg[i] == SEG_OUTPUT;
             double m = -INFINITY;
             for (int j = 0; j < S; ++j) {
                 if (!use[j / B]) continue;
-                double s = raw_score(qr, k + ((size_t)h * S + j) * d, d, inv_sqrt_d);
+                double s = qk8 != NULL ? qk8_score(qk8, (size_t)h * S + i, (size_t)h * S + j, d, inv_sqrt_d)
+                                       : raw_score(qr, k + ((size_t)h * S + j) * d, d, inv_sqrt_d);
                 if (biased_row && seg[j] == SEG_GUIDE) {
                     double dt = fabs((double)times[i] - (double)times[j]);
                     s -= oracle_penalty(dt, pen[0], pen[1], pen[2], pen[3]);
@@ -288,6 +305,71 @@ void oracle_attend(int H, int S, int d, int B, const uint8_t *seg, const float *
     }
     free(vid_index);
     free(nonvideo);
+}
+
+void oracle_attend(int H, int S, int d, int B, const uint8_t *seg, const float *times,
+                   const double *pen, const int32_t *sel, int kk, const uint16_t *q,
+                   const uint16_t *k, const uint16_t *v, int n, const int32_t *heads,
+                   const int32_t *rows, double *out_o, double *out_lse) {
+    attend_core(H, S, d, B, seg, times, pen, sel, kk, q, k, v, NULL, n, heads, rows, out_o, out_lse);
+}
+
+/* ---- int8 QK ([SLA] inputs table, use_int8_qk) ----
+ *
+ * Q and K are quantised to int8 per token with a dynamic scale before the
+ * QK dot product; PV stays at the inputs' precision.  Per row x of d values:
+ *   a = max_c |x_c|,  s = a / 127,  code_c = clamp(rint(x_c * (127 / a)), -127, 127);
+ *   a row of zeros gets s = 0 and zero codes.
+ * The page fixes no arithmetic for this; the two quotients and the product
+ * are taken in fp32 with round-to-nearest-even (rint: ties to even), so that
+ * a code is decided the same way wherever the rule is evaluated.  The score
+ * of (query i, key j) becomes s_q,i s_k,j (sum_c code_q,c code_k,c) / sqrt(d);
+ * everything after it (penalty, softmax, PV) is unchanged.
+ */
+static inline float bf16_to_f32(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+void oracle_quantize_rows(long n_rows, int d, const uint16_t *x, int8_t *codes, float *scales) {
+    for (long r = 0; r < n_rows; ++r) {
+        const uint16_t *xr = x + (size_t)r * d;
+        int8_t *cr = codes + (size_t)r * d;
+        float a = 0.0f;
+        for (int c = 0; c < d; ++c) {
+            float m = fabsf(bf16_to_f32(xr[c]));
+            if (m > a) a = m;
+        }
+        if (a == 0.0f) {
+            scales[r] = 0.0f;
+            for (int c = 0; c < d; ++c) cr[c] = 0;
+            continue;
+        }
+        scales[r] = a / 127.0f;
+        float inv = 127.0f / a;
+        for (int c = 0; c < d; ++c) {
+            float t = rintf(bf16_to_f32(xr[c]) * inv);
+            if (t > 127.0f) t = 127.0f;
+            if (t < -127.0f) t = -127.0f;
+            cr[c] = (int8_t)t;
+        }
+    }
+}
+
+/*
+ * As oracle_attend, with the int8 QK score above: q8/k8 are the codes and
+ * sq/sk the scales of Q and K ([H][S][d] and [H][S], from oracle_quantize_rows);
+ * v stays bf16.
+ */
+void oracle_attend_qk8(int H, int S, int d, int B, const uint8_t *seg, const float *times,
+                       const double *pen, const int32_t *sel, int kk, const int8_t *q8,
+                       const float *sq, const int8_t *k8, const float *sk, const uint16_t *v,
+                       int n, const int32_t *heads, const int32_t *rows, double *out_o,
+                       double *out_lse) {
+    qk8_operands o = {q8, k8, sq, sk};
+    attend_core(H, S, d, B, seg, times, pen, sel, kk, NULL, NULL, v, &o, n, heads, rows, out_o, out_lse);
 }
 
 /* ---- Flash-Partitions evaluation of the same rule ([FP §3], [FP §4]) ---- */

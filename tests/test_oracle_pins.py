@@ -396,3 +396,82 @@ def test_tail_term_is_absent_without_dropped_blocks():
     a = oracle.attend(q, k, v, seg, times, pen=None, sel=sel, heads=np.zeros_like(rows), rows=rows)
     b = oracle.attend_tail(q, k, v, seg, times, None, sel, np.zeros_like(rows), rows)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+# ---------------------------------------------------------------- int8 QK --
+# "H3 SLA Attention", inputs table, use_int8_qk: Q and K quantised per token
+# with a dynamic scale before the QK dot product; PV unchanged.
+
+def _bits(vals):
+    return inputs.f32_to_bf16_bits(np.asarray(vals, np.float32))
+
+
+def test_quantize_hand_row():
+    """max |x| = 1: scale 1/127, codes 127 x rounded half to even (63.5 -> 64, -63.5 -> -64)."""
+    x = _bits([[1.0, -0.5, 0.25, 0.125, 0.75, -1.0, 0.0, 0.5]])
+    codes, scales = oracle.quantize_rows(x)
+    assert codes.tolist() == [[127, -64, 32, 16, 95, -127, 0, 64]]
+    assert scales[0] == np.float32(1.0) / np.float32(127.0)
+
+
+def test_quantize_zero_row_and_power_of_two_invariance():
+    x = np.zeros((1, 16), np.uint16)
+    codes, scales = oracle.quantize_rows(x)
+    assert not codes.any() and scales[0] == 0.0
+    rng = np.random.default_rng(3)
+    base = rng.standard_normal((5, 64)).astype(np.float32)
+    c0, s0 = oracle.quantize_rows(_bits(base))
+    for e in (-6, -1, 3, 9):
+        c, s = oracle.quantize_rows(_bits(base * np.float32(2.0 ** e)))
+        assert np.array_equal(c, c0)
+        assert np.array_equal(s, s0 * np.float32(2.0 ** e))
+
+
+def test_quantize_reconstruction_bound():
+    """Every code is within half a step of x / s, and each nonzero row reaches +-127."""
+    rng = np.random.default_rng(5)
+    xb = _bits(rng.standard_normal((200, 128)) * rng.uniform(0.01, 30.0, (200, 1)))
+    codes, scales = oracle.quantize_rows(xb)
+    x = inputs.bf16_bits_to_f64(xb)
+    err = np.abs(x - codes.astype(np.float64) * scales[:, None].astype(np.float64))
+    assert np.all(err <= 0.5 * scales[:, None] * (1 + 1e-5))
+    assert np.all(np.abs(codes).max(axis=1) == 127)
+
+
+def _exact_int8_rows(rng, H, S, d):
+    """bf16 rows code * 2^-7 with integer codes in [-127, 127] and one +-127 per row: the quantiser
+    reproduces them exactly (scale 2^-7)."""
+    c = rng.integers(-127, 128, (H, S, d))
+    c[..., 0] = np.where(rng.random((H, S)) < 0.5, 127, -127)
+    return _bits(c.astype(np.float32) / 128.0), c
+
+
+def test_qk8_attend_equals_exact_on_exactly_quantisable_inputs():
+    """When Q and K are exactly int8 times a per-row scale, the int8 score equals the exact one."""
+    segs = [inputs.Segment(inputs.SEG_TEXT, 40), inputs.Segment(inputs.SEG_GUIDE, 3 * 30, 3),
+            inputs.Segment(inputs.SEG_OUTPUT, 3 * 30, 3)]
+    cfg = inputs.custom(2, 32, segs, seed=8)
+    seg, times, _ = cfg.layout()
+    rng = np.random.default_rng(9)
+    q, cq = _exact_int8_rows(rng, cfg.H, cfg.S, 32)
+    k, ck = _exact_int8_rows(rng, cfg.H, cfg.S, 32)
+    v = inputs.tensor(cfg, 2)
+    q8, sq = oracle.quantize_rows(q)
+    assert np.array_equal(q8, cq) and np.all(sq == np.float32(2.0 ** -7))
+    o8, l8 = oracle.attend_qk8(q, k, v, seg, times, pen=DEF)
+    o, l = oracle.attend(q, k, v, seg, times, pen=DEF)
+    assert np.abs(o8 - o).max() <= 1e-12 and np.abs(l8 - l).max() <= 1e-12
+
+
+def test_qk8_attend_error_against_exact():
+    """Gaussian Q/K/V: the int8 QK outputs stay within a few percent of the exact ones (the page reports
+    about 1 % per layer for its int8 attention)."""
+    segs = [inputs.Segment(inputs.SEG_TEXT, 64), inputs.Segment(inputs.SEG_GUIDE, 4 * 48, 4),
+            inputs.Segment(inputs.SEG_OUTPUT, 4 * 48, 4)]
+    cfg = inputs.custom(2, 128, segs, seed=12, cluster_norm=2.0)
+    seg, times, _ = cfg.layout()
+    q, k, v = (inputs.tensor(cfg, i) for i in range(3))
+    o8, _ = oracle.attend_qk8(q, k, v, seg, times, pen=DEF)
+    o, _ = oracle.attend(q, k, v, seg, times, pen=DEF)
+    rel = np.linalg.norm(o8 - o) / np.linalg.norm(o)
+    assert 0.0 < rel <= 0.03, rel
