@@ -27,6 +27,7 @@ EXPORTS = ("h3attn_plan_init", "h3attn_workspace_bytes", "h3attn_pool", "h3attn_
            "h3attn_forward",
            "h3attn_dense_workspace_bytes", "h3attn_dense_biased", "h3attn_check", "h3attn_selftest_timeout",
            "h3attn_attend_host", "h3attn_merge", "h3attn_tail_workspace_bytes", "h3attn_tail_correct",
+           "h3attn_qk8_workspace_bytes", "h3attn_quantize_qk", "h3attn_forward_qk8",
            "h3attn_strerror")
 
 
@@ -96,6 +97,13 @@ def lib():
         L.h3attn_tail_workspace_bytes.restype = ctypes.c_size_t
         L.h3attn_tail_correct.argtypes = [PP, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, ctypes.c_size_t, _P]
         L.h3attn_tail_correct.restype = ctypes.c_int
+        L.h3attn_qk8_workspace_bytes.argtypes = [PP]
+        L.h3attn_qk8_workspace_bytes.restype = ctypes.c_size_t
+        L.h3attn_quantize_qk.argtypes = [PP, _P, _P, _P, ctypes.c_size_t, _P]
+        L.h3attn_quantize_qk.restype = ctypes.c_int
+        L.h3attn_forward_qk8.argtypes = [PP, _P, _P, _P, _P, _P, ctypes.POINTER(Penalty), _P, _P, _P, _P,
+                                         ctypes.c_size_t, _P, ctypes.c_size_t, _P]
+        L.h3attn_forward_qk8.restype = ctypes.c_int
         L.h3attn_check.argtypes = [_P, _P]
         L.h3attn_check.restype = ctypes.c_int
         L.h3attn_selftest_timeout.argtypes = [_P, ctypes.c_uint32, _P]
@@ -203,6 +211,57 @@ def forward(p: Plan, q, k, v, seg, times, pen=DEFAULT_PENALTY, kv_sel=None, ws=N
     _raise(lib().h3attn_forward(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), seg.data_ptr(),
                                 _dptr(times), ctypes.byref(pn) if pn is not None else None, _dptr(kv_sel),
                                 o.data_ptr(), _dptr(lse_t), ws.data_ptr(), ws.numel(), _stream(stream)), "forward")
+    return o, lse_t
+
+
+def qk8_workspace(p: Plan, device="cuda") -> torch.Tensor:
+    """Scratch of the int8-QK path: codes and per-token scales of Q and K."""
+    n = lib().h3attn_qk8_workspace_bytes(ctypes.byref(p))
+    if n == 0:
+        raise H3Error(EINVAL, "qk8_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def _align256(x: int) -> int:
+    return (x + 255) // 256 * 256
+
+
+def quantize_qk(p: Plan, q, k, qk8_ws=None, stream=None):
+    """Per-token int8 quantisation of Q and K (h3attn_quantize_qk).  Returns views of the scratch:
+    (q8 int8 [H, S, d], k8 int8 [H, S, d], q_scale float32 [H, 64 n_blocks], k_scale float32 [H, 64 n_blocks])."""
+    _check_qkv(q, k, k)
+    if qk8_ws is None:
+        qk8_ws = qk8_workspace(p, q.device)
+    _raise(lib().h3attn_quantize_qk(ctypes.byref(p), q.data_ptr(), k.data_ptr(), qk8_ws.data_ptr(), qk8_ws.numel(),
+                                    _stream(stream)), "quantize_qk")
+    codes = p.H * p.S * p.d
+    stride = p.n_blocks * 64
+    o_k8 = _align256(codes)
+    o_sq = o_k8 + _align256(codes)
+    o_sk = o_sq + _align256(p.H * stride * 4)
+    q8 = qk8_ws[:codes].view(torch.int8).view(p.H, p.S, p.d)
+    k8 = qk8_ws[o_k8:o_k8 + codes].view(torch.int8).view(p.H, p.S, p.d)
+    sq = qk8_ws[o_sq:o_sq + p.H * stride * 4].view(torch.float32).view(p.H, stride)
+    sk = qk8_ws[o_sk:o_sk + p.H * stride * 4].view(torch.float32).view(p.H, stride)
+    return q8, k8, sq, sk
+
+
+def forward_qk8(p: Plan, q, k, v, seg, times, pen=DEFAULT_PENALTY, kv_sel=None, ws=None, qk8_ws=None, out=None,
+                lse: bool | torch.Tensor = False, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """forward with Q and K quantised per token to int8 before the QK product (h3attn_forward_qk8)."""
+    _check_qkv(q, k, v)
+    if ws is None:
+        ws = workspace(p, q.device)
+    if qk8_ws is None:
+        qk8_ws = qk8_workspace(p, q.device)
+    o = torch.empty_like(q) if out is None else out
+    lse_t = lse if isinstance(lse, torch.Tensor) else (
+        torch.empty((p.H, p.S), dtype=torch.float32, device=q.device) if lse else None)
+    pn = _pen(pen)
+    _raise(lib().h3attn_forward_qk8(ctypes.byref(p), q.data_ptr(), k.data_ptr(), v.data_ptr(), seg.data_ptr(),
+                                    _dptr(times), ctypes.byref(pn) if pn is not None else None, _dptr(kv_sel),
+                                    o.data_ptr(), _dptr(lse_t), ws.data_ptr(), ws.numel(), qk8_ws.data_ptr(),
+                                    qk8_ws.numel(), _stream(stream)), "forward_qk8")
     return o, lse_t
 
 

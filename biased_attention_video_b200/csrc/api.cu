@@ -89,13 +89,43 @@ bool make_map(CUtensorMap* m, const void* base, int H, int S, int d) {
 
 bool finite_nonneg(float x) { return std::isfinite(x) && x >= 0.0f; }
 
+// int8 QK scratch: codes of Q and K [H][S][d], then their per-token scales
+// [H][64 n_blocks] (a whole-block stride keeps each head's scales 16-byte
+// aligned; padding rows hold 0)
+struct Qk8Layout {
+  size_t q8, k8, sq, sk, total;
+  int stride;
+};
+Qk8Layout qk8_layout(const h3attn_plan* plan) {
+  Qk8Layout l;
+  l.stride = plan->n_blocks * h3::kBlock;
+  const size_t codes = (size_t)plan->H * plan->S * plan->d;
+  const size_t scales = (size_t)plan->H * l.stride * sizeof(float);
+  l.q8 = 0;
+  l.k8 = align_up(codes);
+  l.sq = l.k8 + align_up(codes);
+  l.sk = l.sq + align_up(scales);
+  l.total = l.sk + align_up(scales);
+  return l;
+}
+
+struct Qk8Operands {
+  const int8_t *q8, *k8;
+  const float *sq, *sk;
+  int stride;
+};
+
+// qk8: int8 Q / K codes and scales (q, k unused then), or null for bf16 Q / K
 int forward_impl(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, const uint16_t* v,
                  const uint8_t* seg, const float* times, const h3attn_penalty* pen, const int32_t* kv_sel,
-                 uint16_t* o, float* lse, void* ws, size_t ws_bytes, size_t ws_needed, cudaStream_t stream) {
+                 uint16_t* o, float* lse, void* ws, size_t ws_bytes, size_t ws_needed, cudaStream_t stream,
+                 const Qk8Operands* qk8 = nullptr) {
   if (!plan_ok(plan)) return H3ATTN_EINVAL;
-  if (!q || !k || !v || !seg || !o) return H3ATTN_EINVAL;
+  if (qk8 == nullptr && (!q || !k)) return H3ATTN_EINVAL;
+  if (!v || !seg || !o) return H3ATTN_EINVAL;
   if (ws == nullptr || ws_bytes < ws_needed) return H3ATTN_EWORKSPACE;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(ws)) return H3ATTN_EALIGN;
+  if ((qk8 == nullptr && (!aligned16(q) || !aligned16(k))) || !aligned16(v) || !aligned16(o) || !aligned16(ws))
+    return H3ATTN_EALIGN;
   if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return H3ATTN_EALIGN;
   bool pen_on = false;
   if (pen != nullptr) {
@@ -106,7 +136,7 @@ int forward_impl(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, 
     if (pen_on && !(pen->falloff > 0.0f)) return H3ATTN_EINVAL;
     if (pen_on && times == nullptr) return H3ATTN_EINVAL;
   }
-  if (h3::attn_smem_bytes(plan->d, plan->n_blocks) > kMaxSmem) return H3ATTN_EUNSUPPORTED;
+  if (h3::attn_smem_bytes(plan->d, plan->n_blocks, qk8 != nullptr) > kMaxSmem) return H3ATTN_EUNSUPPORTED;
   const bool routed = kv_sel != nullptr && plan->n_video_blocks > 0;
 
   h3::AttnParams p{};
@@ -146,9 +176,17 @@ int forward_impl(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, 
   const int n_qtiles = p.n_dense_tiles + p.n_paired_tiles;
 
   CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, q, plan->H, plan->S, plan->d) || !make_map(&tk, k, plan->H, plan->S, plan->d) ||
-      !make_map(&tv, v, plan->H, plan->S, plan->d))
+  if (qk8 != nullptr) {
+    p.q_scale = qk8->sq;
+    p.k_scale = qk8->sk;
+    p.scale_stride = qk8->stride;
+    if (!h3::encode_u8_3d(&tq, qk8->q8, (uint64_t)plan->d, (uint64_t)plan->S, (uint64_t)plan->H, 128, 64) ||
+        !h3::encode_u8_3d(&tk, qk8->k8, (uint64_t)plan->d, (uint64_t)plan->S, (uint64_t)plan->H, 128, 64))
+      return H3ATTN_ECUDA;
+  } else if (!make_map(&tq, q, plan->H, plan->S, plan->d) || !make_map(&tk, k, plan->H, plan->S, plan->d)) {
     return H3ATTN_ECUDA;
+  }
+  if (!make_map(&tv, v, plan->H, plan->S, plan->d)) return H3ATTN_ECUDA;
   if (h3::launch_kv_desc(seg, pen_on ? times : nullptr, plan->S, plan->n_blocks, reinterpret_cast<uint4*>(wsb + wl.desc),
                          reinterpret_cast<float*>(wsb + wl.gtime), reinterpret_cast<uint32_t*>(wsb + wl.slow),
                          stream) != cudaSuccess)
@@ -156,13 +194,26 @@ int forward_impl(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, 
   if (routed && h3::launch_pair(kv_sel, plan->H, plan->n_blocks, plan->first_video_block, plan->k,
                                 reinterpret_cast<uint32_t*>(wsb + wl.pairs), stream) != cudaSuccess)
     return H3ATTN_ECUDA;
-  if (h3::launch_attn(tq, tk, tv, p, n_qtiles * plan->H, stream) != cudaSuccess) return H3ATTN_ECUDA;
+  if (h3::launch_attn(tq, tk, tv, p, n_qtiles * plan->H, stream, qk8 != nullptr) != cudaSuccess) return H3ATTN_ECUDA;
   return H3ATTN_OK;
 }
 
 }  // namespace
 
 namespace h3 {
+bool encode_u8_3d(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2, uint32_t box0,
+                  uint32_t box1) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {dim0, dim1, dim2};
+  cuuint64_t strides[2] = {dim0, dim0 * dim1};
+  cuuint32_t box[3] = {box0, box1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool encode_bf16_3d(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2, uint32_t box0,
                     uint32_t box1) {
   EncodeTiledFn fn = encode_fn();
@@ -392,6 +443,43 @@ int h3attn_tail_correct(const h3attn_plan* plan, const uint16_t* v, const int32_
                       static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return H3ATTN_ECUDA;
   return H3ATTN_OK;
+}
+
+size_t h3attn_qk8_workspace_bytes(const h3attn_plan* plan) {
+  if (!plan_ok(plan)) return 0;
+  return qk8_layout(plan).total;
+}
+
+int h3attn_quantize_qk(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, void* qk8_ws,
+                       size_t qk8_ws_bytes, void* stream) {
+  if (!plan_ok(plan) || q == nullptr || k == nullptr) return H3ATTN_EINVAL;
+  const Qk8Layout l = qk8_layout(plan);
+  if (qk8_ws == nullptr || qk8_ws_bytes < l.total) return H3ATTN_EWORKSPACE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(qk8_ws)) return H3ATTN_EALIGN;
+  uint8_t* b = static_cast<uint8_t*>(qk8_ws);
+  if (h3::launch_quant_qk(q, k, reinterpret_cast<int8_t*>(b + l.q8), reinterpret_cast<int8_t*>(b + l.k8),
+                          reinterpret_cast<float*>(b + l.sq), reinterpret_cast<float*>(b + l.sk), plan->H, plan->S,
+                          plan->d, l.stride, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return H3ATTN_ECUDA;
+  return H3ATTN_OK;
+}
+
+int h3attn_forward_qk8(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                       const uint8_t* seg, const float* times, const h3attn_penalty* pen, const int32_t* kv_sel,
+                       uint16_t* o, float* lse, void* ws, size_t ws_bytes, void* qk8_ws, size_t qk8_ws_bytes,
+                       void* stream) {
+  if (!plan_ok(plan)) return H3ATTN_EINVAL;
+  if (plan->d != 128) return H3ATTN_EUNSUPPORTED;
+  if (kv_sel != nullptr && (reinterpret_cast<uintptr_t>(kv_sel) & 3u)) return H3ATTN_EALIGN;
+  const int rc = h3attn_quantize_qk(plan, q, k, qk8_ws, qk8_ws_bytes, stream);
+  if (rc != H3ATTN_OK) return rc;
+  const Qk8Layout l = qk8_layout(plan);
+  const uint8_t* b = static_cast<const uint8_t*>(qk8_ws);
+  const Qk8Operands ops{reinterpret_cast<const int8_t*>(b + l.q8), reinterpret_cast<const int8_t*>(b + l.k8),
+                        reinterpret_cast<const float*>(b + l.sq), reinterpret_cast<const float*>(b + l.sk), l.stride};
+  const size_t need = kStatusBytes + attn_scratch_bytes(plan->n_blocks) + (kv_sel != nullptr ? pair_bytes(plan) : 0);
+  return forward_impl(plan, q, k, v, seg, times, pen, kv_sel, o, lse, ws, ws_bytes, need,
+                      static_cast<cudaStream_t>(stream), &ops);
 }
 
 size_t h3attn_dense_workspace_bytes(int S) {

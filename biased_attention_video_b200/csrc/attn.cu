@@ -65,14 +65,18 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 
 __device__ __forceinline__ void report(int* status, int code) { atomicCAS(status, 0, code); }
 
-template <int D>
+template <int D, bool kQK8>
 struct Layout {
-  static constexpr int kHalves = D / 64;               // 128-byte swizzle atoms along d
-  static constexpr int kHalfBytes = kTileRows * 128;   // one d-half of a 128-row tile
+  static constexpr int kHalves = D / 64;               // 128-byte swizzle atoms along d (bf16 V)
+  static constexpr int kHalfBytes = kTileRows * 128;   // one 128-byte-wide column of a 128-row tile
   static constexpr int kTileBytes = kHalves * kHalfBytes;
+  // Q and K: bf16, or int8 codes (one 128-byte atom holds d = 128)
+  static constexpr int kQKHalves = kQK8 ? D / 128 : D / 64;
+  static constexpr int kQKElems = kQK8 ? 128 : 64;  // elements per 128-byte atom
+  static constexpr int kQKTileBytes = kQKHalves * kHalfBytes;
   static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kTileBytes;
-  static constexpr int kV = kK + kTileBytes;
+  static constexpr int kK = kQ + kQKTileBytes;
+  static constexpr int kV = kK + kQKTileBytes;
   // phase-1 probabilities: two K-major 32-byte-swizzled operands (one per key
   // block of the tile), 128 rows x 16 keys each
   static constexpr int kPh1 = kV + kTileBytes;
@@ -230,6 +234,24 @@ __device__ __forceinline__ float fast_offset(const BlockMode& bm, int c0, float 
   return bm.mode == 0 ? -INFINITY : -(m + (c0 < bm.split ? bm.pen_a : bm.pen_b));
 }
 
+// Int8 QK: N raw s32 scores (exact integer dot products of the codes, |s| <
+// 2^22 for d = 128) to fp32 by the exponent trick (2^23 + 2^22 + s is exact
+// in fp32, and its bits are those of the integer plus a constant), times the
+// keys' scales ks[0..N) (16-byte aligned).
+template <int N>
+__device__ __forceinline__ void qk8_scores(const uint32_t* raw, const float* ks, float* out) {
+  constexpr int kMagicBits = 0x4B400000;     // 12582912.0f = 2^23 + 2^22
+  constexpr float kMagic = 12582912.0f;
+#pragma unroll
+  for (int i = 0; i < N; i += 4) {
+    const float4 s = __ldg(reinterpret_cast<const float4*>(ks + i));
+    out[i] = (__int_as_float((int)raw[i] + kMagicBits) - kMagic) * s.x;
+    out[i + 1] = (__int_as_float((int)raw[i + 1] + kMagicBits) - kMagic) * s.y;
+    out[i + 2] = (__int_as_float((int)raw[i + 2] + kMagicBits) - kMagic) * s.z;
+    out[i + 3] = (__int_as_float((int)raw[i + 3] + kMagicBits) - kMagic) * s.w;
+  }
+}
+
 // Maximum over N keys of a fully valid block (-inf if the row skips it).
 template <int N>
 __device__ __forceinline__ float full_max(const float* s, const BlockMode& bm) {
@@ -266,11 +288,15 @@ __device__ __forceinline__ float part_max(const float* s, const BlockMode& bm, i
   return pmax;
 }
 
-template <int D>
+// kQK8: Q and K arrive as int8 codes with per-token scales (p.q_scale,
+// p.k_scale); S = Q K^T runs as int8 MMAs into s32 and is scaled back per
+// query row and key in the softmax.
+template <int D, bool kQK8>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
-  using L = Layout<D>;
+  static_assert(!kQK8 || D == 128, "int8 QK needs d = 128 (one 128-byte atom per row)");
+  using L = Layout<D, kQK8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const Bars bars = carve_bars(smem + L::kBars);
@@ -415,22 +441,22 @@ __global__ void __launch_bounds__(kThreads, 2)
       uint8_t* sq = smem + L::kQ;
       uint8_t* sk = smem + L::kK;
       uint8_t* sv = smem + L::kV;
-      mbar_arrive_expect_tx(bars.q_full, L::kTileBytes);
+      mbar_arrive_expect_tx(bars.q_full, L::kQKTileBytes);
 #pragma unroll
-      for (int c = 0; c < L::kHalves; ++c) {
-        tma_load_3d(sq + c * L::kHalfBytes, &tm_q, bars.q_full, c * 64, qa_row, head);
-        tma_load_3d(sq + c * L::kHalfBytes + 8192, &tm_q, bars.q_full, c * 64, qb_row, head);
+      for (int c = 0; c < L::kQKHalves; ++c) {
+        tma_load_3d(sq + c * L::kHalfBytes, &tm_q, bars.q_full, c * L::kQKElems, qa_row, head);
+        tma_load_3d(sq + c * L::kHalfBytes + 8192, &tm_q, bars.q_full, c * L::kQKElems, qb_row, head);
       }
       for (int j = 0; j < n_tiles; ++j) {
         const uint32_t ph = (uint32_t)j & 1u;
         const int r0 = (int)(list[2 * j] & 0x3FFFu) * 64;
         const int r1 = (2 * j + 1 < n_entries) ? (int)(list[2 * j + 1] & 0x3FFFu) * 64 : oob_row;
         if (!wait_bar(bars.k_empty, ph ^ 1u, p, abort_flag)) break;
-        mbar_arrive_expect_tx(bars.k_full, L::kTileBytes);
+        mbar_arrive_expect_tx(bars.k_full, L::kQKTileBytes);
 #pragma unroll
-        for (int c = 0; c < L::kHalves; ++c) {
-          tma_load_3d(sk + c * L::kHalfBytes, &tm_k, bars.k_full, c * 64, r0, head);
-          tma_load_3d(sk + c * L::kHalfBytes + 8192, &tm_k, bars.k_full, c * 64, r1, head);
+        for (int c = 0; c < L::kQKHalves; ++c) {
+          tma_load_3d(sk + c * L::kHalfBytes, &tm_k, bars.k_full, c * L::kQKElems, r0, head);
+          tma_load_3d(sk + c * L::kHalfBytes + 8192, &tm_k, bars.k_full, c * L::kQKElems, r1, head);
         }
         ++issued_k;
         if (!wait_bar(bars.v_empty, ph ^ 1u, p, abort_flag)) break;
@@ -448,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (issued_v) drain_wait(bars.v_full, (issued_v - 1) & 1u, p);
     } else if (warp == 1 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
-      constexpr uint32_t kIdescS = idesc_bf16_f32(128, kTileKeys, 0, 0);
+      constexpr uint32_t kIdescS = kQK8 ? idesc_s8_s32(128, kTileKeys) : idesc_bf16_f32(128, kTileKeys, 0, 0);
       constexpr uint32_t kIdescO = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t q_addr = smem_u32(smem + L::kQ);
       const uint32_t k_addr = smem_u32(smem + L::kK);
@@ -459,12 +485,16 @@ __global__ void __launch_bounds__(kThreads, 2)
       auto issue_s = [&](int j) -> bool {
         if (!wait_bar(bars.k_full, (uint32_t)j & 1u, p, abort_flag)) return false;
         tc_fence_after();
+        // one MMA per 32-byte K step: 16 bf16 or 32 int8 elements of d
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < L::kQKHalves * 4; ++kk) {
           const int c = kk >> 2, off = (kk & 3) * 32;
           const uint64_t adesc = sw128_desc(q_addr + c * L::kHalfBytes + off, 16, 1024);
           const uint64_t bdesc = sw128_desc(k_addr + c * L::kHalfBytes + off, 16, 1024);
-          umma_ss(tmem_s, adesc, bdesc, kIdescS, kk > 0 ? 1u : 0u);
+          if constexpr (kQK8)
+            umma_ss_i8(tmem_s, adesc, bdesc, kIdescS, kk > 0 ? 1u : 0u);
+          else
+            umma_ss(tmem_s, adesc, bdesc, kIdescS, kk > 0 ? 1u : 0u);
         }
         umma_commit(bars.s_full);
         umma_commit(bars.k_empty);
@@ -540,7 +570,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     const bool row_valid = (r < 64 ? has_a : has_b) && qrow < p.S;
     const bool pen_row = p.pen_on && row_valid && p.seg[qrow] == kSegOutput;
     const float tq = pen_row ? p.times[qrow] : 0.0f;
-    const float scale = p.scale_log2;
+    // log2-units multiplier of this row's scores; with int8 QK it also
+    // carries the row's quantisation scale (the key's is applied per score)
+    const float scale = kQK8 ? (row_valid ? p.q_scale[(size_t)head * p.scale_stride + qrow] : 0.0f) * p.scale_log2
+                             : p.scale_log2;
+    const float* kscale_head = kQK8 ? p.k_scale + (size_t)head * p.scale_stride : nullptr;
     float m = -INFINITY;  // running max, log2 units (upper bound of the true max)
     float l = 0.0f;       // partial row sum over this thread's keys
     bool ok = true;
@@ -657,12 +691,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         tmem_ld16(t_s + 32, t16);
         tmem_ld16(t_s + kPhase0Keys, u16);
         tmem_wait_ld();
+        if constexpr (kQK8) {
+          const float* ks = kscale_head + bm.key0;
+          qk8_scores<32>(t32, ks, sv);
+          qk8_scores<16>(t16, ks + 32, sv + 32);
+          qk8_scores<16>(u16, ks + kPhase0Keys, sv1);
+        } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) sv[i] = __uint_as_float(t32[i]);
+          for (int i = 0; i < 32; ++i) sv[i] = __uint_as_float(t32[i]);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) sv[32 + i] = __uint_as_float(t16[i]);
+          for (int i = 0; i < 16; ++i) sv[32 + i] = __uint_as_float(t16[i]);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) sv1[i] = __uint_as_float(u16[i]);
+          for (int i = 0; i < 16; ++i) sv1[i] = __uint_as_float(u16[i]);
+        }
       }
       float mx;
       const float pmax = kGeneral ? fmaxf(part_max<kPhase0Keys>(sv, bm, 0), part_max<16>(sv1, bm, kPhase0Keys))
@@ -692,8 +733,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         __syncwarp();
         tmem_ld16(t_s + kPhase0Keys, t16);
         tmem_wait_ld();
+        if constexpr (kQK8) {
+          qk8_scores<16>(t16, kscale_head + bm.key0 + kPhase0Keys, sv1);
+        } else {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) sv1[i] = __uint_as_float(t16[i]);
+          for (int i = 0; i < 16; ++i) sv1[i] = __uint_as_float(t16[i]);
+        }
       }
       // O is stable once PV(j-1, phase 1) has completed (waited on every tile)
       if (j > 0) {
@@ -778,23 +823,28 @@ __global__ void __launch_bounds__(kThreads, 2)
 
 }  // namespace
 
-int attn_smem_bytes(int d, int n_blocks) {
-  return d == 64 ? Layout<64>::host_bytes(n_blocks) : Layout<128>::host_bytes(n_blocks);
+int attn_smem_bytes(int d, int n_blocks, bool qk8) {
+  if (qk8) return Layout<128, true>::host_bytes(n_blocks);
+  return d == 64 ? Layout<64, false>::host_bytes(n_blocks) : Layout<128, false>::host_bytes(n_blocks);
 }
 
-cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                        const AttnParams& p, int n_ctas, cudaStream_t stream) {
-  const int smem = attn_smem_bytes(p.d, p.n_blocks);
-  if (p.d == 64) {
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    attn_kernel<64><<<n_ctas, kThreads, smem, stream>>>(tq, tk, tv, p);
-  } else {
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    attn_kernel<128><<<n_ctas, kThreads, smem, stream>>>(tq, tk, tv, p);
-  }
+namespace {
+template <int D, bool kQK8>
+cudaError_t launch_attn_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnParams& p,
+                          int n_ctas, cudaStream_t stream) {
+  const int smem = Layout<D, kQK8>::host_bytes(p.n_blocks);
+  cudaError_t e = cudaFuncSetAttribute(attn_kernel<D, kQK8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  attn_kernel<D, kQK8><<<n_ctas, kThreads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                        const AttnParams& p, int n_ctas, cudaStream_t stream, bool qk8) {
+  if (qk8) return p.d == 128 ? launch_attn_t<128, true>(tq, tk, tv, p, n_ctas, stream) : cudaErrorInvalidValue;
+  return p.d == 64 ? launch_attn_t<64, false>(tq, tk, tv, p, n_ctas, stream)
+                   : launch_attn_t<128, false>(tq, tk, tv, p, n_ctas, stream);
 }
 
 }  // namespace h3

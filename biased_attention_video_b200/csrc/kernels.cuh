@@ -28,6 +28,11 @@ struct AttnParams {
   // n_paired_tiles read from qpairs[H][n_paired_tiles] (see launch_pair)
   const uint32_t* qpairs;
   int n_dense_tiles, n_paired_tiles;
+  // int8 QK (attn kernel instantiated for it): per-token scales of Q and K,
+  // [H][scale_stride] with scale_stride = 64 n_blocks (padding rows 0)
+  const float* q_scale;
+  const float* k_scale;
+  int scale_stride;
   uint16_t* o;                 // bf16 [H][S][d]
   float* lse;                  // [H][S] or null
   int* status;                 // device status word
@@ -38,9 +43,21 @@ struct AttnParams {
   uint64_t wait_ns;            // bounded waits: time budget
 };
 
-int attn_smem_bytes(int d, int n_blocks);
+int attn_smem_bytes(int d, int n_blocks, bool qk8 = false);
+// qk8: tq / tk map int8 Q / K codes ({d, S, H} bytes, box {d, 64}) and the QK
+// products run as int8 MMAs (d = 128 only)
 cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                        const AttnParams& p, int n_ctas, cudaStream_t stream);
+                        const AttnParams& p, int n_ctas, cudaStream_t stream, bool qk8 = false);
+
+// per-token int8 quantisation of Q and K (quant.cu): codes [H][S][d], scales
+// [H][stride] (rows S..stride-1 get 0)
+cudaError_t launch_quant_qk(const uint16_t* q, const uint16_t* k, int8_t* q8, int8_t* k8, float* sq, float* sk,
+                            int H, int S, int d, int stride, cudaStream_t stream);
+
+// int8 tensor [dim2][dim1][dim0] as a 3-D TMA map with a {box0, box1, 1} box
+// and 128-byte swizzle (box0 <= 128)
+bool encode_u8_3d(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2, uint32_t box0,
+                  uint32_t box1);
 
 // kv_desc[b] for every key block b, over its valid rows (n of them):
 //   x = n | kind << 8 | split << 16, y / z = time bits of runs a / b

@@ -244,6 +244,36 @@ H3ATTN_API int h3attn_tail_correct(const h3attn_plan* plan, const uint16_t* v, c
                                    float* lse, void* ws, size_t ws_bytes, void* tail_ws, size_t tail_ws_bytes,
                                    void* stream);
 
+/* Int8 QK ("H3 SLA Attention", inputs table, use_int8_qk: Q and K quantised
+ * to int8 per token with a dynamic scale before the QK dot product on the
+ * selected blocks; PV stays at full precision).
+ *
+ * h3attn_quantize_qk: per row x (d values) of Q and of K,
+ *   a = max|x|,  s = a / 127,  code = clamp(rint(x * (127 / a)), -127, 127),
+ * in fp32 with round-to-nearest-even (ties to even); a zero row gets s = 0 and
+ * zero codes.  q, k: bf16 [H][S][d] device, 16-byte aligned.  qk8_ws: device
+ * scratch of h3attn_qk8_workspace_bytes(plan) bytes, 16-byte aligned (about
+ * 1.7 GB at S = 116,883, H = 56, d = 128), laid out as int8 codes of Q
+ * [H][S][d], int8 codes of K [H][S][d], float32 scales of Q [H][64 n_blocks],
+ * float32 scales of K [H][64 n_blocks], each part starting on a 256-byte
+ * boundary (scale rows S .. 64 n_blocks - 1 hold 0); every call rewrites it.
+ *
+ * h3attn_forward_qk8: h3attn_quantize_qk, then the attention of
+ * h3attn_forward with the score of (query i, key j) taken as
+ * s_q,i s_k,j (sum over d of the codes' products) / sqrt(d), accumulated exactly
+ * in int32 on the tensor cores; penalty, softmax and PV (bf16 V) unchanged.
+ * d must be 128 (H3ATTN_EUNSUPPORTED otherwise).  Other arguments, outputs and
+ * workspace as for h3attn_forward.  The result differs from h3attn_forward's
+ * by the quantisation (about 1 % relative on Gaussian inputs, the scale the
+ * page reports for int8 attention). */
+H3ATTN_API size_t h3attn_qk8_workspace_bytes(const h3attn_plan* plan);
+H3ATTN_API int h3attn_quantize_qk(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, void* qk8_ws,
+                                  size_t qk8_ws_bytes, void* stream);
+H3ATTN_API int h3attn_forward_qk8(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                  const uint8_t* seg, const float* times, const h3attn_penalty* pen,
+                                  const int32_t* kv_sel, uint16_t* o, float* lse, void* ws, size_t ws_bytes,
+                                  void* qk8_ws, size_t qk8_ws_bytes, void* stream);
+
 /* Merge of normalised partition results ("Flash Partitions for H3 native
  * temporal alignment", section 4 "Why log-sum-exp is necessary"): partition i
  * is an attention output O_i over some key set (normalised by its own sum)

@@ -351,6 +351,7 @@ void oracle_quantize_rows(long n_rows, int d, const uint16_t *x, int8_t *codes, 
         float inv = 127.0f / a;
         for (int c = 0; c < d; ++c) {
             float t = rintf(bf16_to_f32(xr[c]) * inv);
+            if (t != t) t = 0.0f; /* 0 * inf when 127 / a overflows (a tiny subnormal max) */
             if (t > 127.0f) t = 127.0f;
             if (t < -127.0f) t = -127.0f;
             cr[c] = (int8_t)t;

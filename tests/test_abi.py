@@ -149,3 +149,21 @@ def test_plan_k_matches_oracle_for_decimal_sparsities():
         assert p.n_video_blocks == nv
         assert p.k == oracle.k_for(nv, sp), (nv, sp, p.k)
     assert h3.plan(1, 64 + 2100 * 64, 64, np.array([0] * 64 + [4] * 2100 * 64, np.uint8), sparsity=0.9).k == 210
+
+
+def test_qk8_validation_before_any_device_work():
+    L = h3.lib()
+    fake = 1 << 40  # never dereferenced: validation fails first
+    seg = np.array([0] * 64 + [4] * 192, np.uint8)
+    p64 = h3.plan(1, 256, 64, seg, sparsity=0.5)
+    need = L.h3attn_qk8_workspace_bytes(ctypes.byref(p64))
+    assert need >= 2 * 256 * 64 + 2 * 256 * 4
+    assert L.h3attn_forward_qk8(ctypes.byref(p64), fake, fake, fake, fake, None, None, None, fake, None, fake,
+                                1 << 30, fake, need, None) == h3.EUNSUPPORTED
+    p = h3.plan(1, 256, 128, seg, sparsity=0.5)
+    need = L.h3attn_qk8_workspace_bytes(ctypes.byref(p))
+    assert L.h3attn_quantize_qk(ctypes.byref(p), None, fake, fake, need, None) == h3.EINVAL
+    assert L.h3attn_quantize_qk(ctypes.byref(p), fake, fake, fake, need - 1, None) == h3.EWORKSPACE
+    assert L.h3attn_quantize_qk(ctypes.byref(p), fake + 2, fake, fake, need, None) == h3.EALIGN
+    assert L.h3attn_forward_qk8(ctypes.byref(p), fake, fake, fake, fake, None, None, None, fake, None, fake,
+                                1 << 30, fake, 16, None) == h3.EWORKSPACE
