@@ -437,9 +437,46 @@ def run_ours(args, rank, world, local_rank):
             raise RuntimeError("device status after the tail correction")
         del lse_t, tail_ws
 
+    # int8 QK (h3attn_forward_qk8: per-token quantisation of Q and K, then the attention with int8 QK
+    # products) at full size on this call's routed lists, and its deviation from the bf16 path's O
+    qk8_ms = quant_ms = float("nan")
+    qk8_rel = None
+    if not args.no_qk8 and d == 128:
+        qws = h3.qk8_workspace(p, dev)
+        o8 = torch.empty_like(o)
+        h3.route(p, qd, kd, ws, kv_sel=sel)
+        for _ in range(2):
+            h3.forward_qk8(p, qd, kd, vd, seg_d, times_d, pen=pen, kv_sel=sel, ws=ws, qk8_ws=qws, out=o8)
+        q0 = torch.cuda.Event(enable_timing=True)
+        q1 = torch.cuda.Event(enable_timing=True)
+        q0.record(stream)
+        for _ in range(args.steps):
+            h3.forward_qk8(p, qd, kd, vd, seg_d, times_d, pen=pen, kv_sel=sel, ws=ws, qk8_ws=qws, out=o8)
+        q1.record(stream)
+        q0b = torch.cuda.Event(enable_timing=True)
+        q1b = torch.cuda.Event(enable_timing=True)
+        q0b.record(stream)
+        for _ in range(args.steps):
+            h3.quantize_qk(p, qd, kd, qws)
+        q1b.record(stream)
+        torch.cuda.synchronize(dev)
+        qk8_ms = q0.elapsed_time(q1) / args.steps
+        quant_ms = q0b.elapsed_time(q1b) / args.steps
+        if h3.check(ws) != h3.OK:
+            raise RuntimeError("device status after the int8 QK call")
+        h3.forward(p, qd, kd, vd, seg_d, times_d, pen=pen, kv_sel=sel, ws=ws, out=o)
+        num = den = 0.0
+        for hh in range(H):
+            a = o8[hh].float()
+            b = o[hh].float()
+            num += float(torch.sum((a - b) ** 2))
+            den += float(torch.sum(b * b))
+        qk8_rel = (num / den) ** 0.5
+        del qws, o8
+
     # max over ranks; with head sharding the job's work is the sum of the ranks' shares
-    ms, e2e_ms, fwd_ms, route_ms, merge_ms, tail_ms = max_over_ranks(
-        [ms, e2e_ms, fwd_ms, route_ms, merge_ms, tail_ms], world, dev)
+    ms, e2e_ms, fwd_ms, route_ms, merge_ms, tail_ms, qk8_ms, quant_ms = max_over_ranks(
+        [ms, e2e_ms, fwd_ms, route_ms, merge_ms, tail_ms, qk8_ms, quant_ms], world, dev)
     local_flops, local_mma = eff_flops, mma_pairs
     if sharded:
         eff_flops, mma_pairs = sum_over_ranks([eff_flops, mma_pairs], world, dev)
@@ -482,7 +519,15 @@ def run_ours(args, rank, world, local_rank):
         "tail": None if args.no_tail else {
             "kernels": "pool_vt, tail_weights, tail_gemm (tcgen05), tail_merge (h3attn_tail_correct)",
             "ms": tail_ms, "share_of_call": tail_ms / ms_step},
-        "gpu_launches": 5 * args.steps,  # pool_split, score_gemm, topk, kv_desc, attn
+        "qk8": None if (args.no_qk8 or d != 128) else {
+            "what": "h3attn_forward_qk8 on the same routed call: per-token int8 quantisation of Q and K "
+                    "(quant_rows_kernel) + attn_kernel with int8 QK MMAs; not the headline (reduced precision)",
+            "ms": qk8_ms, "quantize_ms": quant_ms,
+            "effective_tflops": (local_flops if sharded else eff_flops) / (qk8_ms * 1e-3) / 1e12,
+            "vs_bf16_forward": fwd_ms / qk8_ms,
+            "quantize_gbs": (2 * H * S * d * 3 + 2 * H * p.n_blocks * 64 * 4) / (quant_ms * 1e-3) / 1e9,
+            "rel_fro_vs_bf16": qk8_rel},
+        "gpu_launches": 6 * args.steps,  # pool_split, score_gemm, topk, kv_desc, pair, attn
         "clocks": clk,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms / args.steps},
@@ -514,6 +559,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-merge", action="store_true", help="skip the partition-merge measurement")
     ap.add_argument("--no-tail", action="store_true", help="skip the pooled-tail-term measurement")
+    ap.add_argument("--no-qk8", action="store_true", help="skip the int8-QK measurement")
     ap.add_argument("--shard", choices=["none", "heads"], default="none",
                     help="N>1: 'none' = one independent call per GPU (weak scaling); 'heads' = one call, its heads "
                          "split over the GPUs (strong scaling)")

@@ -241,14 +241,18 @@ __device__ __forceinline__ float fast_offset(const BlockMode& bm, int c0, float 
 template <int N>
 __device__ __forceinline__ void qk8_scores(const uint32_t* raw, const float* ks, float* out) {
   constexpr int kMagicBits = 0x4B400000;     // 12582912.0f = 2^23 + 2^22
-  constexpr float kMagic = 12582912.0f;
+  const uint64_t magic2 = f2_pack(12582912.0f, 12582912.0f);
 #pragma unroll
   for (int i = 0; i < N; i += 4) {
     const float4 s = __ldg(reinterpret_cast<const float4*>(ks + i));
-    out[i] = (__int_as_float((int)raw[i] + kMagicBits) - kMagic) * s.x;
-    out[i + 1] = (__int_as_float((int)raw[i + 1] + kMagicBits) - kMagic) * s.y;
-    out[i + 2] = (__int_as_float((int)raw[i + 2] + kMagicBits) - kMagic) * s.z;
-    out[i + 3] = (__int_as_float((int)raw[i + 3] + kMagicBits) - kMagic) * s.w;
+    const uint64_t a = f2_mul(f2_sub(f2_pack(__int_as_float((int)raw[i] + kMagicBits),
+                                             __int_as_float((int)raw[i + 1] + kMagicBits)), magic2),
+                              f2_pack(s.x, s.y));
+    const uint64_t b = f2_mul(f2_sub(f2_pack(__int_as_float((int)raw[i + 2] + kMagicBits),
+                                             __int_as_float((int)raw[i + 3] + kMagicBits)), magic2),
+                              f2_pack(s.z, s.w));
+    f2_unpack(a, out[i], out[i + 1]);
+    f2_unpack(b, out[i + 2], out[i + 3]);
   }
 }
 
@@ -574,7 +578,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     // carries the row's quantisation scale (the key's is applied per score)
     const float scale = kQK8 ? (row_valid ? p.q_scale[(size_t)head * p.scale_stride + qrow] : 0.0f) * p.scale_log2
                              : p.scale_log2;
-    const float* kscale_head = kQK8 ? p.k_scale + (size_t)head * p.scale_stride : nullptr;
     float m = -INFINITY;  // running max, log2 units (upper bound of the true max)
     float l = 0.0f;       // partial row sum over this thread's keys
     bool ok = true;
@@ -692,7 +695,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         tmem_ld16(t_s + kPhase0Keys, u16);
         tmem_wait_ld();
         if constexpr (kQK8) {
-          const float* ks = kscale_head + bm.key0;
+          const float* ks = p.k_scale + ((size_t)head * p.scale_stride + bm.key0);
           qk8_scores<32>(t32, ks, sv);
           qk8_scores<16>(t16, ks + 32, sv + 32);
           qk8_scores<16>(u16, ks + kPhase0Keys, sv1);
@@ -734,7 +737,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         tmem_ld16(t_s + kPhase0Keys, t16);
         tmem_wait_ld();
         if constexpr (kQK8) {
-          qk8_scores<16>(t16, kscale_head + bm.key0 + kPhase0Keys, sv1);
+          qk8_scores<16>(t16, p.k_scale + ((size_t)head * p.scale_stride + bm.key0 + kPhase0Keys), sv1);
         } else {
 #pragma unroll
           for (int i = 0; i < 16; ++i) sv1[i] = __uint_as_float(t16[i]);
