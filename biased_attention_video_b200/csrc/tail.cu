@@ -102,10 +102,10 @@ __global__ void __launch_bounds__(256) tail_weights_kernel(const float* __restri
   __syncwarp();
   const float* srow = scores + (size_t)row * ldc;
   const int last_rows = S - (first_block + n_video - 1) * kBlock;  // valid rows of the last block
+  const float log_full = __logf((float)kBlock), log_last = __logf((float)last_rows);
   auto logit = [&](int j) -> float {  // s_ij + log n_j of a dropped block, -inf for a routed one
     if ((kept[j >> 5] >> (j & 31)) & 1u) return -INFINITY;
-    const float nj = j == n_video - 1 ? (float)last_rows : (float)kBlock;
-    return fmaf(srow[j], scale, __logf(nj));
+    return fmaf(srow[j], scale, j == n_video - 1 ? log_last : log_full);
   };
   float m = -INFINITY;
   for (int j = lane; j < n_video; j += 32) m = fmaxf(m, logit(j));

@@ -166,6 +166,19 @@ def test_forward_routed_paired_groups(sparsity):
     assert p.first_video_block == 3 and p.n_blocks == 101
 
 
+@pytest.mark.parametrize("segs,fvb,nb", [
+    (_layout(0, 0, 4, 200, 5, 230), 0, 31),        # all video: every tile is a paired one
+    (_layout(100, 30, 0, 0, 1, 150), 3, 5),        # video block 3 in the mixed dense tile, block 4 alone
+    (_layout(128, 0, 0, 0, 1, 40), 2, 3),          # one video block after an even prefix: a lone tile
+    (_layout(64, 0, 0, 0, 1, 40), 1, 2),           # one video block inside the dense tile (0, 1)
+    (_layout(70, 0, 1, 60, 1, 100), 2, 4),         # 70 prefix rows: video blocks 2 and 3 paired
+])
+def test_forward_routed_pairing_edges(segs, fvb, nb):
+    cfg = inputs.custom(2, 64, segs, seed=57, cluster_norm=2.0)
+    _, p = _forward_all_rows(cfg, 0.5, PEN, routed=True)
+    assert p.first_video_block == fvb and p.n_blocks == nb
+
+
 def test_config1_dense_biased():
     cfg = inputs.CONFIGS[1]
     x = make(cfg)
