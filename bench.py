@@ -32,7 +32,6 @@ sys.path.insert(0, ROOT)
 
 import inputs  # noqa: E402
 
-CONFIG_ID = 5
 WORKLOAD = "full combined: S=116883 (text 256|image-ref 1013|audio 810|guide 27x2126|output 27x2126), " \
            "H=56, d=128, bf16, block 64, sparsity 0.90 (k=180 of 1794 video KV blocks), default penalty"
 
@@ -254,7 +253,7 @@ def run_reference(args, rank, world):
     """Reference arm: the fp64 CPU oracle, rank 0 only."""
     if rank != 0:
         return
-    cfg = inputs.CONFIGS[CONFIG_ID]
+    cfg = inputs.FULL_COMBINED
     seg, times, _ = cfg.layout()
     small = inputs.custom(1, cfg.d, cfg.segments, cfg.seed, cluster_norm=cfg.cluster_norm)
     q, k, v = (inputs.tensor(small, t) for t in range(3))
@@ -286,7 +285,7 @@ def run_ours(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    cfg = inputs.CONFIGS[CONFIG_ID]
+    cfg = inputs.FULL_COMBINED
     if args.heads is not None:
         cfg = inputs.custom(args.heads, cfg.d, cfg.segments, cfg.seed, cluster_norm=cfg.cluster_norm,
                             penalty=cfg.penalty, sparsities=cfg.sparsities, name=f"{cfg.name} ({args.heads} heads)")

@@ -137,6 +137,9 @@ CONFIGS = {
               seed=1005, cluster_norm=2.0, penalty=DEFAULT_PENALTY, sparsities=(0.90,)),
 }
 
+# the benchmark's workload: the full routed, penalised call
+FULL_COMBINED = CONFIGS[5]
+
 
 def custom(H: int, d: int, segments: Sequence[Segment], seed: int, cluster_norm: float = 0.0,
            penalty=None, sparsities=(0.0,), name: str = "custom") -> Config:
