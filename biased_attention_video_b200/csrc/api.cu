@@ -135,6 +135,7 @@ int forward_impl(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, 
     pen_on = pen->strength > 0.0f && pen->cap > 0.0f;
     if (pen_on && !(pen->falloff > 0.0f)) return H3ATTN_EINVAL;
     if (pen_on && times == nullptr) return H3ATTN_EINVAL;
+    if (pen_on && (reinterpret_cast<uintptr_t>(times) & 3u)) return H3ATTN_EALIGN;
   }
   if (h3::attn_smem_bytes(plan->d, plan->n_blocks, qk8 != nullptr) > kMaxSmem) return H3ATTN_EUNSUPPORTED;
   const bool routed = kv_sel != nullptr && plan->n_video_blocks > 0;
@@ -534,7 +535,7 @@ const char* h3attn_strerror(int status) {
     case H3ATTN_OK: return "ok";
     case H3ATTN_EINVAL: return "invalid argument";
     case H3ATTN_EUNSUPPORTED: return "unsupported shape or layout";
-    case H3ATTN_EALIGN: return "pointer not aligned (16 bytes for tensors and workspace)";
+    case H3ATTN_EALIGN: return "pointer not aligned (16 bytes for tensors and workspace, 4 for int32/float32 arrays)";
     case H3ATTN_ECUDA: return "CUDA call or kernel launch failed";
     case H3ATTN_ETIMEOUT: return "a bounded device-side wait gave up";
     case H3ATTN_EWORKSPACE: return "workspace missing or too small";

@@ -37,8 +37,9 @@
  * Conventions for every call:
  *  - Q, K, V, O are bf16 (passed as uint16_t bit patterns), layout
  *    [H][S][d], contiguous, row-major, on the device; base addresses 16-byte
- *    aligned.  seg is uint8 [S] and times is float32 [S] (seconds), on the
- *    device; times are read only for guide/output rows.
+ *    aligned.  seg is uint8 [S] and times is float32 [S] (seconds, 4-byte
+ *    aligned), on the device; times are read only for guide/output rows.
+ *    Integer and float32 arrays (kv_sel, lse, times) need 4-byte alignment.
  *  - The caller owns every buffer; the library allocates no memory.
  *  - All device work is asynchronous on `stream` (a cudaStream_t; NULL = the
  *    legacy default stream).  Only h3attn_check synchronises.
@@ -67,7 +68,7 @@ extern "C" {
 #define H3ATTN_OK 0
 #define H3ATTN_EINVAL (-1)       /* bad argument: null pointer, bad size, bad value */
 #define H3ATTN_EUNSUPPORTED (-2) /* d not 64/128, block not 64, video rows not a suffix, S too large */
-#define H3ATTN_EALIGN (-3)       /* a base address is not 16-byte aligned */
+#define H3ATTN_EALIGN (-3)       /* a base address is misaligned (16 bytes for tensors, 4 for int32/float32 arrays) */
 #define H3ATTN_ECUDA (-4)        /* a CUDA runtime/driver call or launch failed */
 #define H3ATTN_ETIMEOUT (-5)     /* a bounded device-side wait gave up */
 #define H3ATTN_EWORKSPACE (-6)   /* workspace missing or too small */

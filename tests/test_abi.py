@@ -107,6 +107,14 @@ def test_host_validation_before_any_device_work():
                             None) == h3.EWORKSPACE
     assert L.h3attn_forward(ctypes.byref(p), fake + 2, fake, fake, fake, fake, None, None, fake, None, fake,
                             ws_need, None) == h3.EALIGN
+    pen = h3.Penalty(*h3.DEFAULT_PENALTY)
+    # times is read as float32 when the penalty is on; kv_sel as int32
+    assert L.h3attn_forward(ctypes.byref(p), fake, fake, fake, fake, fake + 2, ctypes.byref(pen), None, fake, None,
+                            fake, ws_need, None) == h3.EALIGN
+    assert L.h3attn_forward(ctypes.byref(p), fake, fake, fake, fake, fake, ctypes.byref(pen), fake + 2, fake, None,
+                            fake, ws_need, None) == h3.EALIGN
+    assert L.h3attn_forward(ctypes.byref(p), fake, fake, fake, fake, fake, None, None, fake, fake + 1, fake,
+                            ws_need, None) == h3.EALIGN
     bad_pen = h3.Penalty(2.0, 0.2, 0.0, 6.0)  # falloff 0 with the penalty on
     assert L.h3attn_forward(ctypes.byref(p), fake, fake, fake, fake, fake, ctypes.byref(bad_pen), None, fake, None,
                             fake, ws_need, None) == h3.EINVAL
