@@ -188,9 +188,9 @@ int forward_impl(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, 
     return H3ATTN_ECUDA;
   }
   if (!make_map(&tv, v, plan->H, plan->S, plan->d)) return H3ATTN_ECUDA;
-  if (h3::launch_kv_desc(seg, pen_on ? times : nullptr, plan->S, plan->n_blocks, reinterpret_cast<uint4*>(wsb + wl.desc),
-                         reinterpret_cast<float*>(wsb + wl.gtime), reinterpret_cast<uint32_t*>(wsb + wl.slow),
-                         stream) != cudaSuccess)
+  if (h3::launch_kv_desc(seg, pen_on ? times : nullptr, plan->S, plan->n_blocks,
+                         reinterpret_cast<uint4*>(wsb + wl.desc), reinterpret_cast<float*>(wsb + wl.gtime),
+                         reinterpret_cast<uint32_t*>(wsb + wl.slow), stream) != cudaSuccess)
     return H3ATTN_ECUDA;
   if (routed && h3::launch_pair(kv_sel, plan->H, plan->n_blocks, plan->first_video_block, plan->k,
                                 reinterpret_cast<uint32_t*>(wsb + wl.pairs), stream) != cudaSuccess)
