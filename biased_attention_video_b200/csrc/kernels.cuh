@@ -54,6 +54,12 @@ cudaError_t launch_attn(const CUtensorMap& tq, const CUtensorMap& tk, const CUte
 cudaError_t launch_quant_qk(const uint16_t* q, const uint16_t* k, int8_t* q8, int8_t* k8, float* sq, float* sk,
                             int H, int S, int d, int stride, cudaStream_t stream);
 
+// float32 tensor [dim2][dim1][pitch] (dim0 <= pitch valid columns, pitch a
+// multiple of 4) as a 3-D TMA map with a {box0, box1, 1} box and 128-byte
+// swizzle (box0 = 32)
+bool encode_f32_3d(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2, uint64_t pitch,
+                   uint32_t box0, uint32_t box1);
+
 // int8 tensor [dim2][dim1][dim0] as a 3-D TMA map with a {box0, box1, 1} box
 // and 128-byte swizzle (box0 <= 128)
 bool encode_u8_3d(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2, uint32_t box0,

@@ -107,25 +107,41 @@ __global__ void __launch_bounds__(256) pool_split_kernel(const uint16_t* __restr
 
 
 // ----------------------------------------------------------- score GEMM
-constexpr int kGemmThreads = 128;
+// Persistent: one CTA per SM walks the 128 x 256 output tiles (head, query
+// blocks, key blocks) in steps of the grid size.  Warp 0 loads 64-element K
+// chunks of A and B through a three-stage TMA ring, warp 1 issues the MMAs into
+// one of two TMEM accumulators (2 x 256 columns), and warps 2..5 write the
+// other accumulator's scores out, so the epilogue of tile i overlaps the MMAs
+// of tile i + 1.  Each epilogue warp stages 32 rows x 32 scores in shared
+// memory (128-byte swizzle, two buffers) and stores them with one TMA tile
+// store, which also drops the rows and columns past the video blocks.  The
+// scores' HBM writes bound it (4 B per score).
+constexpr int kGemmThreads = 192;
 constexpr int kGM = 128;                    // query blocks per tile (UMMA M)
 constexpr int kGN = 256;                    // key blocks per tile (UMMA N)
-constexpr int kGStages = 2;
+constexpr int kGStages = 3;
 constexpr int kGStageA = kGM * 128;         // one 64-element (128-byte) K chunk of A
 constexpr int kGStageB = kGN * 128;
 constexpr int kGStageBytes = kGStageA + kGStageB;
-constexpr int kGBars = kGStages * kGStageBytes;
-constexpr int kGSmem = 1024 + kGBars + 64;
+constexpr int kGEpi = kGStages * kGStageBytes;  // epilogue staging: 4 warps x 2 x 4 KB
+constexpr int kGEpiBytes = 4 * 2 * 4096;
+constexpr int kGBars = kGEpi + kGEpiBytes;
+constexpr int kGNumBars = 2 * kGStages + 5;  // full, empty, acc_full[2], acc_empty[2], drain
+constexpr int kGSmem = 1024 + kGBars + kGNumBars * 8 + 16;
+constexpr uint32_t kGTmemCols = 2 * kGN;
 
-__device__ __forceinline__ bool gemm_wait(uint64_t* bar, uint32_t parity, int* status) {
+// Bounded wait with CTA-wide abort (on give-up: abort flag and status word).
+__device__ __forceinline__ bool gemm_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* status) {
   uint64_t t0 = 0;
   for (uint32_t i = 0;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
     if ((i & 1023u) == 1023u) {
       uint64_t now;
       asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
       if (t0 == 0) t0 = now;
       if (now - t0 > 2000000000ull) {
+        *abort = 1;
         if (status != nullptr) atomicCAS(status, 0, kStatusTimeout);
         return false;
       }
@@ -133,102 +149,182 @@ __device__ __forceinline__ bool gemm_wait(uint64_t* bar, uint32_t parity, int* s
   }
 }
 
-// scores[h][i][j] (row pitch ldc floats) for query blocks i in [m0, m0 + 128)
-// and key blocks j in [n0, n0 + 256) of head h.  Rows past n_video read as
-// zero (TMA fill) and are not stored.
-__global__ void __launch_bounds__(kGemmThreads, 2)
+// Bounded wait for in-flight async work before exit (ignores the abort flag).
+__device__ __forceinline__ void gemm_drain(uint64_t* bar, uint32_t parity, int* status) {
+  uint64_t t0 = 0;
+  for (uint32_t i = 0;; ++i) {
+    if (mbar_try_wait(bar, parity)) return;
+    if ((i & 1023u) == 1023u) {
+      uint64_t now;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
+      if (t0 == 0) t0 = now;
+      if (now - t0 > 2000000000ull) {
+        if (status != nullptr) atomicCAS(status, 0, kStatusTimeout);
+        return;
+      }
+    }
+  }
+}
+
+// scores[h][i][j] for every video query block i and video key block j of
+// every head, written through tm_c (fp32 [H][n_video] rows of pitch ldc, TMA
+// store map).  Tile t covers head t / (n_tm n_tn), query blocks
+// [128 ((t / n_tn) % n_tm), +128) and key blocks [256 (t % n_tn), +256); rows
+// past n_video read as zero (TMA fill) and are not stored.
+__global__ void __launch_bounds__(kGemmThreads, 1)
     score_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                      float* __restrict__ scores, int n_video, int ldc, int n_chunks, int* status) {
+                      const __grid_constant__ CUtensorMap tm_c, int n_video, int n_chunks, int n_tm, int n_tn,
+                      int n_tiles, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kGBars);
   uint64_t* empty = full + kGStages;
-  uint64_t* done = empty + kGStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* acc_full = empty + kGStages;  // [2]: accumulator b holds a finished tile
+  uint64_t* acc_empty = acc_full + 2;     // [2]: the epilogue has read accumulator b
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n0 = blockIdx.x * kGN, m0 = blockIdx.y * kGM, h = blockIdx.z;
   if (tid == 0) {
     for (int s = 0; s < kGStages; ++s) {
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
     }
-    mbar_init(done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(acc_full + b, 1);
+      mbar_init(acc_empty + b, 4);  // one arrival per epilogue warp
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_a);
     tma_prefetch_desc(&tm_b);
+    tma_prefetch_desc(&tm_c);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 256);
+    tmem_alloc(tmem_slot, kGTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const int per_head = n_tm * n_tn;
 
-  if (warp == 0 && lane == 0) {
-    uint32_t issued[kGStages] = {0, 0};
-    for (int c = 0; c < n_chunks; ++c) {
-      const int s = c % kGStages;
-      const uint32_t ph = (uint32_t)(c / kGStages) & 1u;
-      if (!gemm_wait(empty + s, ph ^ 1u, status)) break;
-      uint8_t* st = smem + s * kGStageBytes;
-      mbar_arrive_expect_tx(full + s, kGStageBytes);
-      tma_load_3d(st, &tm_a, full + s, c * 64, m0, h);
-      tma_load_3d(st + kGStageA, &tm_b, full + s, c * 64, n0, h);
-      ++issued[s];
-    }
-    for (int s = 0; s < kGStages; ++s)
-      if (issued[s]) gemm_wait(full + s, (issued[s] - 1) & 1u, status);
-  } else if (warp == 1 && lane == 0) {
-    constexpr uint32_t kIdesc = idesc_bf16_f32(kGM, kGN, 0, 0);
-    for (int c = 0; c < n_chunks; ++c) {
-      const int s = c % kGStages;
-      const uint32_t ph = (uint32_t)(c / kGStages) & 1u;
-      if (!gemm_wait(full + s, ph, status)) break;
-      tc_fence_after();
-      const uint32_t a = smem_u32(smem + s * kGStageBytes), b = a + kGStageA;
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        umma_ss(tmem, sw128_desc(a + kk * 32, 16, 1024), sw128_desc(b + kk * 32, 16, 1024), kIdesc,
-                (c > 0 || kk > 0) ? 1u : 0u);
-      umma_commit(empty + s);
-    }
-    umma_commit(done);
-  }
-  // epilogue: thread = query block row; TMEM -> fp32 scores
-  const bool got = gemm_wait(done, 0, status);
-  if (__all_sync(0xFFFFFFFFu, got)) {
-    tc_fence_after();
-    const int i = m0 + warp * 32 + lane;
-    float* row = scores + ((size_t)h * n_video + (i < n_video ? i : 0)) * ldc;
-#pragma unroll 1
-    for (int cc = 0; cc < kGN / 32; ++cc) {
-      uint32_t v[32];
-      __syncwarp();
-      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + cc * 32, v);
-      tmem_wait_ld();
-      const int j0 = n0 + cc * 32;
-      if (i < n_video && j0 < n_video) {
-        if (j0 + 32 <= n_video) {
-          float4* dst = reinterpret_cast<float4*>(row + j0);
-#pragma unroll
-          for (int t = 0; t < 8; ++t)
-            dst[t] = make_float4(__uint_as_float(v[4 * t]), __uint_as_float(v[4 * t + 1]), __uint_as_float(v[4 * t + 2]),
-                                 __uint_as_float(v[4 * t + 3]));
-        } else {
-#pragma unroll
-          for (int t = 0; t < 32; ++t)
-            if (j0 + t < n_video) row[j0 + t] = __uint_as_float(v[t]);
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- producer
+      uint32_t issued[kGStages] = {};
+      uint32_t q = 0;  // K chunks issued so far, over all tiles
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+        const int h = t / per_head, m0 = ((t / n_tn) % n_tm) * kGM, n0 = (t % n_tn) * kGN;
+        for (int c = 0; c < n_chunks; ++c, ++q) {
+          const int s = (int)(q % kGStages);
+          const uint32_t ph = (q / kGStages) & 1u;
+          if (!gemm_wait(empty + s, ph ^ 1u, abort_flag, status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * kGStageBytes;
+          mbar_arrive_expect_tx(full + s, kGStageBytes);
+          tma_load_3d(st, &tm_a, full + s, c * 64, m0, h);
+          tma_load_3d(st + kGStageA, &tm_b, full + s, c * 64, n0, h);
+          ++issued[s];
         }
       }
+      // every issued load lands before the CTA may exit
+      for (int s = 0; s < kGStages; ++s)
+        if (issued[s]) gemm_drain(full + s, (issued[s] - 1) & 1u, status);
     }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      constexpr uint32_t kIdesc = idesc_bf16_f32(kGM, kGN, 0, 0);
+      uint32_t q = 0;
+      bool ok = true;
+      int i = 0;  // tiles of this CTA so far
+      for (int t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++i) {
+        const int b = i & 1;
+        // accumulator b is free once the epilogue has read its previous tile
+        if (!gemm_wait(acc_empty + b, ((uint32_t)(i >> 1) & 1u) ^ 1u, abort_flag, status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(b * kGN);
+        for (int c = 0; c < n_chunks; ++c, ++q) {
+          const int s = (int)(q % kGStages);
+          const uint32_t ph = (q / kGStages) & 1u;
+          if (!gemm_wait(full + s, ph, abort_flag, status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a = smem_u32(smem + s * kGStageBytes), bb = a + kGStageA;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_ss(d_tmem, sw128_desc(a + kk * 32, 16, 1024), sw128_desc(bb + kk * 32, 16, 1024), kIdesc,
+                    (c > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(empty + s);
+        }
+        if (ok) umma_commit(acc_full + b);
+      }
+      // every issued MMA completes before TMEM is released
+      umma_commit(drain);
+      gemm_drain(drain, 0, status);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    // thread = query block row (TMEM lane); warp w reads lanes 32 (w % 4)..
+    // and writes each 32 x 32 block of scores through shared memory: row r at
+    // byte 128 r, its 16-byte chunk c at chunk c ^ (r & 7) (the 128-byte
+    // swizzle of the store's tensor map; conflict-free for the warp)
+    const int quarter = warp & 3;
+    const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+    uint8_t* stage = smem + kGEpi + (warp - 2) * 2 * 4096;
+    uint32_t n_st = 0;  // 32 x 32 blocks staged by this warp
+    int i = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
+      const int b = i & 1;
+      if (!__all_sync(0xFFFFFFFFu, gemm_wait(acc_full + b, (uint32_t)(i >> 1) & 1u, abort_flag, status))) break;
+      tc_fence_after();
+      const int h = t / per_head, m0 = ((t / n_tn) % n_tm) * kGM, n0 = (t % n_tn) * kGN;
+      const int row0 = m0 + quarter * 32;
+#pragma unroll 1
+      for (int cc = 0; cc < kGN / 32; ++cc) {
+        uint32_t v[32];
+        __syncwarp();
+        tmem_ld32(tmem + lane_addr + (uint32_t)(b * kGN + cc * 32), v);
+        tmem_wait_ld();
+        const int j0 = n0 + cc * 32;
+        if (row0 >= n_video || j0 >= n_video) continue;  // warp-uniform: nothing of the block is stored
+        uint8_t* buf = stage + (n_st & 1u) * 4096;
+        // the store that read this buffer two blocks ago is done with it
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
+        uint8_t* my_row = buf + lane * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(my_row + ((c ^ (lane & 7)) << 4)) =
+              make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+        fence_proxy_async_smem();  // generic-proxy writes -> visible to the bulk store
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&tm_c, buf, j0, row0, h);
+          bulk_commit();
+        }
+        ++n_st;
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty + b);
+    }
+    // every store has written global memory before the CTA exits
+    if (lane == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, kGTmemCols);
   }
 }
 
@@ -512,8 +608,18 @@ cudaError_t launch_route_pipeline(const uint16_t* q, const uint16_t* k, int32_t*
     return cudaErrorInvalidValue;
   e = cudaFuncSetAttribute(score_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmem);
   if (e != cudaSuccess) return e;
-  dim3 ggrid((n_video + kGN - 1) / kGN, (n_video + kGM - 1) / kGM, H);
-  score_gemm_kernel<<<ggrid, kGemmThreads, kGSmem, stream>>>(ta, tb, sc, n_video, (int)r.ldc, 3 * d / 64, status);
+  int dev = 0, n_sm = 0;
+  e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const int n_tm = (n_video + kGM - 1) / kGM, n_tn = (n_video + kGN - 1) / kGN;
+  const long long tiles = (long long)H * n_tm * n_tn;
+  if (tiles > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  const int ggrid = (int)(tiles < n_sm ? tiles : n_sm);
+  CUtensorMap tc;
+  if (!encode_f32_3d(&tc, sc, n_video, n_video, H, r.ldc, 32, 32)) return cudaErrorInvalidValue;
+  score_gemm_kernel<<<ggrid, kGemmThreads, kGSmem, stream>>>(ta, tb, tc, n_video, 3 * d / 64, n_tm, n_tn, (int)tiles,
+                                                             status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // 3. top-k per (head, query block): scores in registers up to 2048 video
