@@ -107,38 +107,36 @@ class Config:
 DEFAULT_PENALTY = (2.0, 0.20, 0.25, 6.0)   # strength, window [s], falloff [s], cap
 
 # The five workloads of the hot path (packings as stated for the H3 call).
-CONFIGS = {
-    # tiny dense biased: text 64 | audio 160 | guide 8x112 | output 8x116
-    1: Config("tiny dense biased S=2048 H=2 d=64", H=2, d=64,
-              segments=(Segment(SEG_TEXT, 64), Segment(SEG_AUDIO, 160),
-                        Segment(SEG_GUIDE, 896, 8), Segment(SEG_OUTPUT, 928, 8)),
-              seed=1001, penalty=DEFAULT_PENALTY, sparsities=(0.0,)),
-    # routing-only: text 256 | audio 384 | video 41 frames x 384
-    2: Config("routing S=16384 H=8 d=128 s=0.85", H=8, d=128,
-              segments=(Segment(SEG_TEXT, 256), Segment(SEG_AUDIO, 384),
-                        Segment(SEG_OUTPUT, 15744, 41)),
-              seed=1002, cluster_norm=2.0, sparsities=(0.85,)),
-    # mid clip: text 256 | image-ref 1024 | audio 400 | video 24 frames x 1978
-    3: Config("mid clip S=49152 H=56 d=128", H=56, d=128,
-              segments=(Segment(SEG_TEXT, 256), Segment(SEG_IMAGE_REF, 1024),
-                        Segment(SEG_AUDIO, 400), Segment(SEG_OUTPUT, 47472, 24)),
-              seed=1003, cluster_norm=2.0, sparsities=(0.0, 0.60, 0.85, 0.90)),
-    # full dense biased: text 256 | image-ref 1013 | audio 810 | guide 27x2126 | output 27x2126
-    4: Config("full dense biased S=116883 H=56 d=128", H=56, d=128,
-              segments=(Segment(SEG_TEXT, 256), Segment(SEG_IMAGE_REF, 1013),
-                        Segment(SEG_AUDIO, 810), Segment(SEG_GUIDE, 57402, 27),
-                        Segment(SEG_OUTPUT, 57402, 27)),
-              seed=1004, cluster_norm=2.0, penalty=DEFAULT_PENALTY, sparsities=(0.0,)),
-    # full combined: as 4, routed to the top 10 % of video KV blocks, penalty on
-    5: Config("full combined S=116883 H=56 d=128 s=0.90", H=56, d=128,
-              segments=(Segment(SEG_TEXT, 256), Segment(SEG_IMAGE_REF, 1013),
-                        Segment(SEG_AUDIO, 810), Segment(SEG_GUIDE, 57402, 27),
-                        Segment(SEG_OUTPUT, 57402, 27)),
-              seed=1005, cluster_norm=2.0, penalty=DEFAULT_PENALTY, sparsities=(0.90,)),
-}
+# tiny dense biased: text 64 | audio 160 | guide 8x112 | output 8x116
+TINY_DENSE = Config("tiny dense biased S=2048 H=2 d=64", H=2, d=64,
+                    segments=(Segment(SEG_TEXT, 64), Segment(SEG_AUDIO, 160),
+                              Segment(SEG_GUIDE, 896, 8), Segment(SEG_OUTPUT, 928, 8)),
+                    seed=1001, penalty=DEFAULT_PENALTY, sparsities=(0.0,))
+# routing-only: text 256 | audio 384 | video 41 frames x 384
+ROUTING_ONLY = Config("routing S=16384 H=8 d=128 s=0.85", H=8, d=128,
+                      segments=(Segment(SEG_TEXT, 256), Segment(SEG_AUDIO, 384),
+                                Segment(SEG_OUTPUT, 15744, 41)),
+                      seed=1002, cluster_norm=2.0, sparsities=(0.85,))
+# mid clip: text 256 | image-ref 1024 | audio 400 | video 24 frames x 1978
+MID_CLIP = Config("mid clip S=49152 H=56 d=128", H=56, d=128,
+                  segments=(Segment(SEG_TEXT, 256), Segment(SEG_IMAGE_REF, 1024),
+                            Segment(SEG_AUDIO, 400), Segment(SEG_OUTPUT, 47472, 24)),
+                  seed=1003, cluster_norm=2.0, sparsities=(0.0, 0.60, 0.85, 0.90))
+# full dense biased: text 256 | image-ref 1013 | audio 810 | guide 27x2126 | output 27x2126
+FULL_DENSE = Config("full dense biased S=116883 H=56 d=128", H=56, d=128,
+                    segments=(Segment(SEG_TEXT, 256), Segment(SEG_IMAGE_REF, 1013),
+                              Segment(SEG_AUDIO, 810), Segment(SEG_GUIDE, 57402, 27),
+                              Segment(SEG_OUTPUT, 57402, 27)),
+                    seed=1004, cluster_norm=2.0, penalty=DEFAULT_PENALTY, sparsities=(0.0,))
+# full combined (the benchmark's workload): the full dense packing, routed to
+# the top 10 % of video KV blocks, penalty on
+FULL_COMBINED = Config("full combined S=116883 H=56 d=128 s=0.90", H=56, d=128,
+                       segments=(Segment(SEG_TEXT, 256), Segment(SEG_IMAGE_REF, 1013),
+                                 Segment(SEG_AUDIO, 810), Segment(SEG_GUIDE, 57402, 27),
+                                 Segment(SEG_OUTPUT, 57402, 27)),
+                       seed=1005, cluster_norm=2.0, penalty=DEFAULT_PENALTY, sparsities=(0.90,))
 
-# the benchmark's workload: the full routed, penalised call
-FULL_COMBINED = CONFIGS[5]
+WORKLOADS = (TINY_DENSE, ROUTING_ONLY, MID_CLIP, FULL_DENSE, FULL_COMBINED)
 
 
 def custom(H: int, d: int, segments: Sequence[Segment], seed: int, cluster_norm: float = 0.0,

@@ -40,9 +40,8 @@ def test_library_targets_sm100a():
     assert "sm_100a" in out
 
 
-@pytest.mark.parametrize("c", [1, 2, 3, 4, 5])
-def test_plan_matches_oracle_block_classes(c):
-    cfg = inputs.CONFIGS[c]
+@pytest.mark.parametrize("cfg", inputs.WORKLOADS, ids=lambda c: c.name)
+def test_plan_matches_oracle_block_classes(cfg):
     seg, _, _ = cfg.layout()
     for s in cfg.sparsities:
         p = h3.plan(cfg.H, cfg.S, cfg.d, seg, sparsity=s)
@@ -56,11 +55,11 @@ def test_plan_matches_oracle_block_classes(c):
 
 
 def test_plan_known_values():
-    seg5, _, _ = inputs.CONFIGS[5].layout()
-    p = h3.plan(56, 116883, 128, seg5, sparsity=0.90)
+    seg_full, _, _ = inputs.FULL_COMBINED.layout()
+    p = h3.plan(56, 116883, 128, seg_full, sparsity=0.90)
     assert (p.n_blocks, p.first_video_block, p.n_video_blocks, p.k, p.prefix_rows) == (1827, 33, 1794, 180, 2079)
-    seg2, _, _ = inputs.CONFIGS[2].layout()
-    p2 = h3.plan(8, 16384, 128, seg2, sparsity=0.85)
+    seg_r, _, _ = inputs.ROUTING_ONLY.layout()
+    p2 = h3.plan(8, 16384, 128, seg_r, sparsity=0.85)
     assert (p2.n_blocks, p2.first_video_block, p2.n_video_blocks, p2.k) == (256, 10, 246, 37)
 
 

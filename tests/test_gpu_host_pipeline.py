@@ -58,8 +58,8 @@ def _case(cfg, sparsity, pen, chunk_heads, same_stream=False):
 
 
 @pytest.mark.parametrize("chunk_heads", [1, 3, 8])
-def test_host_pipeline_config2_routed(chunk_heads):
-    cfg = inputs.CONFIGS[2]
+def test_host_pipeline_routing_only(chunk_heads):
+    cfg = inputs.ROUTING_ONLY
     x, p, got, sel = _case(cfg, 0.85, None, chunk_heads)
     # and a few rows against the oracle
     heads, rows = [0, cfg.H - 1], np.array([0, 700, 5000, 16383])

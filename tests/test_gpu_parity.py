@@ -59,13 +59,13 @@ def _route_and_compare(cfg, sparsity, heads=None):
     return p, x, sel, ws
 
 
-def test_route_config2():
-    _route_and_compare(inputs.CONFIGS[2], 0.85)
+def test_route_routing_only():
+    _route_and_compare(inputs.ROUTING_ONLY, 0.85)
 
 
 @pytest.mark.parametrize("sparsity", [0.0, 0.60, 0.85, 0.90])
-def test_route_config3_sampled_heads(sparsity):
-    _route_and_compare(inputs.CONFIGS[3], sparsity, heads=[0, 27, 55])
+def test_route_mid_clip_sampled_heads(sparsity):
+    _route_and_compare(inputs.MID_CLIP, sparsity, heads=[0, 27, 55])
 
 
 def test_route_more_than_2048_video_blocks():
@@ -179,8 +179,8 @@ def test_forward_routed_pairing_edges(segs, fvb, nb):
     assert p.first_video_block == fvb and p.n_blocks == nb
 
 
-def test_config1_dense_biased():
-    cfg = inputs.CONFIGS[1]
+def test_tiny_dense_biased():
+    cfg = inputs.TINY_DENSE
     x = make(cfg)
     o, l = h3.dense_biased(x["q_d"], x["k_d"], x["v_d"], x["seg_d"], x["times_d"], pen=PEN, lse=True)
     torch.cuda.synchronize()
@@ -192,9 +192,9 @@ def test_config1_dense_biased():
     _forward_all_rows(cfg, 0.0, PEN, routed=True)
 
 
-def test_peaked_scores_config1():
+def test_peaked_scores_tiny_dense():
     """Q x 4 makes the softmax peaked (max-abs binding), still within tolerance."""
-    cfg = inputs.CONFIGS[1]
+    cfg = inputs.TINY_DENSE
     x = make(cfg, device=None)
     qf = inputs.bf16_bits_to_f64(x["q"]) * 4.0
     q4 = inputs.f32_to_bf16_bits(qf.astype(np.float32)).reshape(x["q"].shape)
@@ -202,7 +202,7 @@ def test_peaked_scores_config1():
                            torch.from_numpy(x["times"]).cuda(), pen=PEN)
     ref_o, _ = oracle.attend(q4, x["k"], x["v"], x["seg"], x["times"], pen=PEN)
     H, S, d = x["q"].shape
-    compare_outputs(host_bits(o).reshape(H * S, d), ref_o, "config 1 peaked")
+    compare_outputs(host_bits(o).reshape(H * S, d), ref_o, "tiny dense peaked")
 
 
 def _sampled_forward(cfg, sparsity, pen, heads, blocks, x=None):
@@ -230,22 +230,21 @@ def _sampled_forward(cfg, sparsity, pen, heads, blocks, x=None):
     return x, p
 
 
-def test_config2_routed():
-    cfg = inputs.CONFIGS[2]
+def test_routing_only_routed():
+    cfg = inputs.ROUTING_ONLY
     _sampled_forward(cfg, 0.85, None, heads=list(range(8)), blocks=[0, 5, 9, 10, 11, 100, 200, 255])
 
 
 @pytest.mark.parametrize("sparsity", [0.0, 0.90])
-def test_config3_sampled(sparsity):
-    cfg = inputs.CONFIGS[3]
+def test_mid_clip_sampled(sparsity):
+    cfg = inputs.MID_CLIP
     _sampled_forward(cfg, sparsity, None, heads=[0, 31, 55], blocks=[0, 25, 26, 27, 28, 300, 600, 767])
 
 
-@pytest.mark.parametrize("c", [4, 5])
-def test_full_size_sampled(c):
+@pytest.mark.parametrize("cfg", [inputs.FULL_DENSE, inputs.FULL_COMBINED], ids=lambda c: c.name)
+def test_full_size_sampled(cfg):
     """S = 116,883, H = 56, d = 128: forced/mixed block 32, first video block 33,
     the guide/output boundary block 929, frame-straddling blocks and the 19-row tail."""
-    cfg = inputs.CONFIGS[c]
     _sampled_forward(cfg, cfg.sparsities[0], PEN, heads=[0, 55],
                      blocks=[0, 31, 32, 33, 34, 100, 500, 928, 929, 930, 1500, 1825, 1826])
 

@@ -90,7 +90,7 @@ def test_forward_qk8_no_penalty_and_close_to_bf16():
 
 def test_forward_qk8_full_size_sampled():
     """S = 116,883, H = 56, d = 128 at sparsity 0.90 with the penalty: sampled rows of two heads."""
-    cfg = inputs.CONFIGS[5]
+    cfg = inputs.FULL_COMBINED
     x = make(cfg)
     p = h3.plan(cfg.H, cfg.S, cfg.d, x["seg"], sparsity=cfg.sparsities[0])
     ws = h3.workspace(p)

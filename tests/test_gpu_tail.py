@@ -34,8 +34,8 @@ def _compare(cfg, x, p, sel, o, lse, pen, heads, rows):
     assert np.abs(lse.cpu().numpy()[heads][:, rows].reshape(-1) - ref_l).max() <= LSE_ABS
 
 
-def test_tail_config2():
-    cfg = inputs.CONFIGS[2]
+def test_tail_routing_only():
+    cfg = inputs.ROUTING_ONLY
     x = make(cfg)
     p, sel, o, lse, o_routed = _run(cfg, x, 0.85, None)
     rows = sample_rows(cfg.S, [0, 9, 10, 11, 100, 200, 255])

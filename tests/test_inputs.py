@@ -5,7 +5,7 @@ import inputs
 
 
 def test_counter_based_rows_match_full_tensor():
-    cfg = inputs.CONFIGS[2]
+    cfg = inputs.ROUTING_ONLY
     small = inputs.custom(3, cfg.d, cfg.segments, cfg.seed, cluster_norm=2.0)
     full = inputs.tensor(small, inputs.TENSOR_K, h0=0, nh=3, row0=600, nrows=300)
     again = inputs.tensor(small, inputs.TENSOR_K, h0=0, nh=3, row0=600, nrows=300)
@@ -43,21 +43,20 @@ def test_cluster_mean_shared_by_frame_and_norm():
     assert np.linalg.norm(q[:64].mean(0)) < 2.0         # prefix rows: no mean (noise ~1.41)
 
 
-def test_config_layouts():
-    for c, S in [(1, 2048), (2, 16384), (3, 49152), (4, 116883), (5, 116883)]:
-        cfg = inputs.CONFIGS[c]
+def test_workload_layouts():
+    for cfg, S in zip(inputs.WORKLOADS, (2048, 16384, 49152, 116883, 116883)):
         seg, times, frame = cfg.layout()
         assert cfg.S == S and len(seg) == S
         video = np.where((seg == 3) | (seg == 4))[0]
         assert video[0] == S - len(video)            # video rows are a contiguous suffix
         assert np.all(times[seg < 3] == 0.0)
-    seg, times, frame = inputs.CONFIGS[5].layout()
+    seg, times, frame = inputs.FULL_COMBINED.layout()
     assert list(np.bincount(seg, minlength=5)) == [256, 1013, 810, 57402, 57402]
     g = np.where(seg == 3)[0]
     o = np.where(seg == 4)[0]
     assert times[g[0]] == 0.0 and abs(times[g[-1]] - 26 * 4 / 24) < 1e-6
     assert np.array_equal(times[g], times[o])     # matching temporal grids
-    seg1, t1, _ = inputs.CONFIGS[1].layout()
+    seg1, t1, _ = inputs.TINY_DENSE.layout()
     assert list(np.bincount(seg1, minlength=5)) == [64, 0, 160, 896, 928]
 
 

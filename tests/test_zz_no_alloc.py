@@ -28,10 +28,9 @@ def _route_static_abi(p, q, k):
 
 @pytest.mark.gpu
 def test_route_static_matches_route_on_consecutive_calls():
-    cfg2 = inputs.CONFIGS[2]
-    c3 = inputs.CONFIGS[3]
-    cfg3 = inputs.custom(8, c3.d, c3.segments, c3.seed, cluster_norm=c3.cluster_norm)
-    for cfg, s in [(cfg2, 0.85), (cfg3, 0.60)]:
+    mid = inputs.MID_CLIP
+    mid8 = inputs.custom(8, mid.d, mid.segments, mid.seed, cluster_norm=mid.cluster_norm)
+    for cfg, s in [(inputs.ROUTING_ONLY, 0.85), (mid8, 0.60)]:
         x = make(cfg)
         p = h3.plan(cfg.H, cfg.S, cfg.d, x["seg"], sparsity=s)
         static_sel = _route_static_abi(p, x["q_d"], x["k_d"])
@@ -44,7 +43,7 @@ def test_route_static_matches_route_on_consecutive_calls():
 
 def test_route_static_rejects_problems_beyond_its_scratch():
     """Checked on the host before any device work: 56 heads x 1794 video blocks x d=128 is too large."""
-    seg, _, _ = inputs.CONFIGS[5].layout()
+    seg, _, _ = inputs.FULL_COMBINED.layout()
     p = h3.plan(56, 116883, 128, seg, sparsity=0.9)
     fake = 1 << 40
     assert h3.lib().h3attn_route_static(ctypes.byref(p), fake, fake, fake, None) == h3.EWORKSPACE
