@@ -221,15 +221,14 @@ def oracle_sample(cfg, q, k, v, seg, times, pen, sparsity, budget_s: float, head
     nkb = (cfg.S + 63) // 64
     cls = oracle.block_classes(seg)
     fvb = int(cls.sum())
+    # the edge blocks first (first and last prefix block, first video block, the
+    # ragged last block), then every other block in a seeded random order; eight
+    # rows of each; the time budget decides how far down the list it gets
     rng = np.random.default_rng(1234)
-    blocks = [0, fvb - 1, fvb, nkb - 1] + list(rng.integers(fvb, nkb, size=64))
+    edge = list(dict.fromkeys(b for b in (0, fvb - 1, fvb, nkb - 1) if 0 <= b < nkb))
+    blocks = edge + [int(b) for b in rng.permutation(nkb) if int(b) not in edge]
     rows_done, flops = 0, 0
-    rows_all = []
-    for b in blocks:
-        for r in (0, 21, 42, 63):
-            x = int(b) * 64 + r
-            if x < cfg.S:
-                rows_all.append(x)
+    rows_all = [b * 64 + r for b in blocks for r in (0, 9, 18, 27, 36, 45, 54, 63) if b * 64 + r < cfg.S]
     rows_per_key = np.minimum(64, cfg.S - np.arange(nkb) * 64)
     forced_keys = int(rows_per_key[:fvb].sum())
     i = 0
