@@ -24,6 +24,7 @@ SEG_TEXT, SEG_IMAGE_REF, SEG_AUDIO, SEG_GUIDE, SEG_OUTPUT = 0, 1, 2, 3, 4
 
 # every symbol the C header declares
 EXPORTS = ("h3attn_plan_init", "h3attn_workspace_bytes", "h3attn_pool", "h3attn_route", "h3attn_route_static",
+           "h3attn_route_static_check",
            "h3attn_forward",
            "h3attn_dense_workspace_bytes", "h3attn_dense_biased", "h3attn_check", "h3attn_selftest_timeout",
            "h3attn_attend_host", "h3attn_merge", "h3attn_tail_workspace_bytes", "h3attn_tail_correct",
@@ -79,6 +80,8 @@ def lib():
         L.h3attn_route.restype = ctypes.c_int
         L.h3attn_route_static.argtypes = [PP, _P, _P, _P, _P]
         L.h3attn_route_static.restype = ctypes.c_int
+        L.h3attn_route_static_check.argtypes = [_P]
+        L.h3attn_route_static_check.restype = ctypes.c_int
         L.h3attn_forward.argtypes = [PP, _P, _P, _P, _P, _P, ctypes.POINTER(Penalty), _P, _P, _P, _P,
                                      ctypes.c_size_t, _P]
         L.h3attn_forward.restype = ctypes.c_int
@@ -196,6 +199,11 @@ def route_static(p: Plan, q: torch.Tensor, k: torch.Tensor, kv_sel=None, stream=
     _raise(lib().h3attn_route_static(ctypes.byref(p), q.data_ptr(), k.data_ptr(), kv_sel.data_ptr(),
                                      _stream(stream)), "route_static")
     return kv_sel
+
+
+def route_static_check(stream=None) -> int:
+    """Synchronise and return (then clear) the status word of the route_static calls on the current device."""
+    return lib().h3attn_route_static_check(_stream(stream))
 
 
 def forward(p: Plan, q, k, v, seg, times, pen=DEFAULT_PENALTY, kv_sel=None, ws=None, out=None,

@@ -10,7 +10,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libh3attn.so")
 SOURCES = ["api.cu", "attn.cu", "pool.cu", "route.cu", "route_static.cu", "merge.cu", "tail.cu", "pair.cu", "quant.cu"]
-HEADERS = ["ptx.cuh", "kernels.cuh", "fastmath.cuh"]
+HEADERS = ["ptx.cuh", "kernels.cuh", "fastmath.cuh", "softmax.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [

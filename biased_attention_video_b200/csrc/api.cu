@@ -19,7 +19,7 @@ constexpr size_t kAlign = 256;
 constexpr size_t kStatusBytes = 256;
 constexpr uint32_t kWaitPolls = 0xFFFFFFFFu;
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait: far above any legitimate stall
-constexpr int kMaxSmem = 227 * 1024;
+using h3::kMaxSmem;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 

@@ -10,6 +10,7 @@ constexpr int kSegGuide = 3;
 constexpr int kSegOutput = 4;
 constexpr int kBlock = 64;
 constexpr int kMaxBlocks = 8192;  // S <= 524288: one 16-bit block id, lists fit in shared memory
+constexpr int kMaxSmem = 227 * 1024;  // opt-in dynamic shared memory of one CTA on sm_100
 
 // device status word values (the C ABI maps them to H3ATTN_E*)
 constexpr int kStatusTimeout = 1;

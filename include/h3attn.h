@@ -158,16 +158,27 @@ H3ATTN_API int h3attn_route(const h3attn_plan* plan, const uint16_t* q, const ui
  * Same result as h3attn_route.  Its scratch (the two-part bf16 pooled
  * centroids of Q and K and the fp32 score matrix) is a fixed 32 MiB array
  * inside the library that every GPU loading the library holds until the
- * process exits; problems needing more, i.e. with
+ * process exits; its first 256 bytes are the status word of these calls, and
+ * problems needing more than the remaining 32 MiB - 256 bytes, i.e. with
  * 12 * H * n_video_blocks * d + 16 * H * n_video_blocks * ceil(n_video_blocks / 4)
- * bytes above about 32 MiB, are rejected with H3ATTN_EWORKSPACE.  Every call overwrites all the scratch
- * it reads, so nothing needs clearing between calls; calls that overlap on the
- * GPU (other streams, other threads) share the array and race.  The first call
- * on a device looks up the array's device address with that device current;
- * make that first call before any stream capture.  Allocates nothing and calls
- * no allocating routine. */
+ * bytes above that, are rejected with H3ATTN_EWORKSPACE.  Every call overwrites
+ * all the scratch it reads, so nothing needs clearing between calls; calls
+ * that overlap on the GPU (other streams, other threads) share the array and
+ * race.  A bounded device-side wait that gives up is recorded in the status
+ * word, not returned: call h3attn_route_static_check to read it.  The array's
+ * device address is looked up on the first call with a device current, and
+ * again when that device's current context has changed (for instance after
+ * cudaDeviceReset); make that first call before any stream capture.
+ * Allocates nothing and calls no allocating routine. */
 H3ATTN_API int h3attn_route_static(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, int32_t* kv_sel,
                                    void* stream);
+
+/* Synchronise `stream`, then return and clear the status word of the
+ * h3attn_route_static calls made on the current device: H3ATTN_OK, or
+ * H3ATTN_ETIMEOUT when a bounded device-side wait of one of them gave up (its
+ * kv_sel is then not valid); H3ATTN_ECUDA if the stream reports an error.
+ * Allocates nothing. */
+H3ATTN_API int h3attn_route_static_check(void* stream);
 
 /* Exact attention over the routed tiles with the temporal penalty.
  * Each query row attends: all keys if its block is a forced (non-video)
