@@ -34,20 +34,31 @@ import inputs  # noqa: E402
 
 WORKLOAD = "full combined: S=116883 (text 256|image-ref 1013|audio 810|guide 27x2126|output 27x2126), " \
            "H=56, d=128, bf16, block 64, sparsity 0.90 (k=180 of 1794 video KV blocks), default penalty"
+WORKLOAD_DENSE = "full dense biased: S=116883 (text 256|image-ref 1013|audio 810|guide 27x2126|output 27x2126), " \
+                 "H=56, d=128, bf16, sparsity 0 (every key), default penalty"
+METRIC = "effective attention TFLOP/s (S=116883, H=56, d=128, sparsity 0.90, penalty on)"
+METRIC_DENSE = "effective attention TFLOP/s (S=116883, H=56, d=128, dense, penalty on)"
 
 
-# DRAM bytes of one attn_kernel launch measured by ncu (dram__bytes_read.sum + dram__bytes_write.sum of an
-# 8-head launch of this packing, profiles/attn_kernel_full_combined_H8.md), scaled by heads.  Valid only for
-# the kernel source it was taken from; reported as null once csrc/attn.cu changes.
+# DRAM bytes of one attn_kernel launch as ncu counted them (dram__bytes_read.sum + dram__bytes_write.sum of one
+# 8-head launch of this packing, captured with --clock-control none), scaled by heads: a stored figure, not a
+# per-run measurement.  Valid only for the kernel sources it was taken from (attn.cu and softmax.cuh, hashed
+# together); reported as null once either changes.
 ATTN_TRAFFIC = {"source_sha256_prefix": "625bc0b48a1fbb0b", "bytes_per_head": (1.441045e9 + 0.231585e9) / 8}
+ATTN_SOURCES = ("attn.cu", "softmax.cuh")
+
+
+def attn_source_digest() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in ATTN_SOURCES:
+        with open(os.path.join(ROOT, "biased_attention_video_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 def attn_traffic_bytes(H: int):
-    import hashlib
-    path = os.path.join(ROOT, "biased_attention_video_b200", "csrc", "attn.cu")
-    with open(path, "rb") as f:
-        digest = hashlib.sha256(f.read()).hexdigest()
-    if not digest.startswith(ATTN_TRAFFIC["source_sha256_prefix"]):
+    if not attn_source_digest().startswith(ATTN_TRAFFIC["source_sha256_prefix"]):
         return None
     return ATTN_TRAFFIC["bytes_per_head"] * H
 
@@ -265,7 +276,7 @@ def run_reference(args, rank, world):
             total_flops += f
             total_s += s
     value = total_flops / total_s / 1e12
-    line = {"metric": "effective attention TFLOP/s (S=116883, H=56, d=128, sparsity 0.90, penalty on)",
+    line = {"metric": METRIC,
             "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded generator)", "impl": "reference",
@@ -276,6 +287,92 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def _time_calls(torch, fn, steps: int, warmup: int, stream) -> float:
+    """Mean CUDA-event time (ms) of `steps` back-to-back calls after `warmup` untimed ones."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def extra_configs(args, h3, dev, stream, host, qd, kd, vd, o):
+    """Configuration 4 (dense biased attention at the full packing, default penalty) and configuration 3 (the
+    mid clip at sparsity 0, 0.60, 0.85, 0.90, no penalty, routing included in the call).  Inputs resident in
+    HBM; each call far above L2 (Q+K+V = 5.0 GB and 2.1 GB)."""
+    import torch
+    peaks, _ = measured_peaks()
+    peak = peaks["bf16_tflops_sustained"]
+    steps, warmup = max(1, min(args.steps, 5)), 3
+    out = {}
+
+    # configuration 4: the full packing, dense; inputs of its own seed into the same buffers
+    cfg = inputs.FULL_DENSE
+    seg, times, _ = cfg.layout()
+    for i, t in enumerate(("q", "k", "v")):
+        inputs.tensor(cfg, i, out=host[t].numpy().view(np.uint16))
+    for src, dst in ((host["q"], qd), (host["k"], kd), (host["v"], vd)):
+        dst.view(torch.int16).view(-1).copy_(src)
+    seg_d = torch.from_numpy(seg).to(dev)
+    times_d = torch.from_numpy(times).to(dev)
+    p = h3.plan(cfg.H, cfg.S, cfg.d, seg)
+    ws = h3.workspace(p, dev)
+    ms = _time_calls(torch, lambda: h3.forward(p, qd, kd, vd, seg_d, times_d, pen=cfg.penalty, ws=ws, out=o),
+                     steps, warmup, stream)
+    if h3.check(ws) != h3.OK:
+        raise RuntimeError("device status after the dense call")
+    flops = 4.0 * cfg.d * cfg.H * cfg.S * cfg.S
+    out["full_dense"] = {
+        "workload": "full dense biased: S=116883 (same packing as the headline), H=56, d=128, bf16, sparsity 0, "
+                    "default penalty on output->guide pairs, seed 1004",
+        "ms_per_call": ms, "effective_tflop_per_call": flops / 1e12, "effective_tflops": flops / (ms * 1e-3) / 1e12,
+        "frac_of_sustained_peak": flops / (ms * 1e-3) / 1e12 / peak, "steps": steps, "warmup": warmup}
+    del ws
+
+    # configuration 3: the mid clip, sparsity sweep (routing + attention per call)
+    cfg = inputs.MID_CLIP
+    seg, times, _ = cfg.layout()
+    q3, k3, v3 = (torch.from_numpy(inputs.tensor(cfg, i).view(np.int16)).to(dev).view(torch.bfloat16)
+                  for i in range(3))
+    seg_d = torch.from_numpy(seg).to(dev)
+    times_d = torch.from_numpy(times).to(dev)
+    o3 = torch.empty_like(q3)
+    sweep = []
+    for s in cfg.sparsities:
+        p = h3.plan(cfg.H, cfg.S, cfg.d, seg, sparsity=s)
+        ws = h3.workspace(p, dev)
+        routed = p.n_video_blocks > 0 and p.k < p.n_video_blocks
+        sel = torch.empty((cfg.H, p.n_video_blocks, p.k), dtype=torch.int32, device=dev) if routed else None
+
+        def call():
+            if routed:
+                h3.route(p, q3, k3, ws, kv_sel=sel)
+            h3.forward(p, q3, k3, v3, seg_d, times_d, pen=None, kv_sel=sel, ws=ws, out=o3)
+
+        ms_call = _time_calls(torch, call, steps, warmup, stream)
+        ms_fwd = _time_calls(torch, lambda: h3.forward(p, q3, k3, v3, seg_d, times_d, pen=None, kv_sel=sel, ws=ws,
+                                                       out=o3), steps, 1, stream)
+        if h3.check(ws) != h3.OK:
+            raise RuntimeError(f"device status after the mid-clip call at sparsity {s}")
+        flops = 4.0 * cfg.d * effective_pairs(p, sel.cpu().numpy() if routed else None)
+        sweep.append({"sparsity": s, "k": int(p.k), "ms_per_call": ms_call, "attention_ms": ms_fwd,
+                      "route_ms": ms_call - ms_fwd if routed else 0.0,
+                      "effective_tflop_per_call": flops / 1e12, "effective_tflops": flops / (ms_call * 1e-3) / 1e12,
+                      "attention_tflops": flops / (ms_fwd * 1e-3) / 1e12,
+                      "attention_frac_of_sustained_peak": flops / (ms_fwd * 1e-3) / 1e12 / peak})
+        del ws, sel
+    out["mid_clip_sweep"] = {"workload": "mid clip: S=49152 (text 256|image-ref 1024|audio 400|video 24x1978), "
+                                         "H=56, d=128, bf16, block 64, no penalty, seed 1003",
+                             "steps": steps, "warmup": warmup, "points": sweep}
+    return out
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -284,7 +381,7 @@ def run_ours(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    cfg = inputs.FULL_COMBINED
+    cfg = inputs.FULL_DENSE if args.workload == "full_dense" else inputs.FULL_COMBINED
     if args.heads is not None:
         cfg = inputs.custom(args.heads, cfg.d, cfg.segments, cfg.seed, cluster_norm=cfg.cluster_norm,
                             penalty=cfg.penalty, sparsities=cfg.sparsities, name=f"{cfg.name} ({args.heads} heads)")
@@ -312,7 +409,8 @@ def run_ours(args, rank, world, local_rank):
     seg_d, times_d = seg_h.to(dev), times_h.to(dev)
     p = h3.plan(H, S, d, seg, sparsity=sparsity)
     ws = h3.workspace(p, dev)
-    sel = torch.empty((H, p.n_video_blocks, p.k), dtype=torch.int32, device=dev)
+    routed = p.n_video_blocks > 0 and p.k < p.n_video_blocks
+    sel = torch.empty((H, p.n_video_blocks, p.k), dtype=torch.int32, device=dev) if routed else None
     o = torch.empty_like(qd)
     stream = torch.cuda.current_stream(dev)
 
@@ -322,7 +420,8 @@ def run_ours(args, rank, world, local_rank):
         if record:
             e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
             e[0].record(stream)
-        h3.route(p, qd, kd, ws, kv_sel=sel)
+        if routed:
+            h3.route(p, qd, kd, ws, kv_sel=sel)
         if record:
             e[1].record(stream)
             e[2].record(stream)
@@ -338,7 +437,7 @@ def run_ours(args, rank, world, local_rank):
     status = h3.check(ws)
     if status != h3.OK:
         raise RuntimeError(f"device status {status} after warm-up")
-    sel_h = sel.cpu().numpy()
+    sel_h = sel.cpu().numpy() if routed else None
     pairs = effective_pairs(p, sel_h)
     eff_flops = 4 * d * pairs
     mma_pairs = executed_mma_pairs(p, sel_h)
@@ -417,7 +516,7 @@ def run_ours(args, rank, world, local_rank):
     # pooled tail term (h3attn_tail_correct) at full size: after route + forward with LSE on this call's
     # inputs; its kernels read V's video rows, the pooled scores, the weights and the O/LSE of video rows
     tail_ms = float("nan")
-    if not args.no_tail and p.n_video_blocks > 0:
+    if not args.no_tail and routed:
         lse_t = torch.empty((H, S), dtype=torch.float32, device=dev)
         tail_ws = h3.tail_workspace(p, dev)
         h3.route(p, qd, kd, ws, kv_sel=sel)
@@ -442,7 +541,8 @@ def run_ours(args, rank, world, local_rank):
     if not args.no_qk8 and d == 128:
         qws = h3.qk8_workspace(p, dev)
         o8 = torch.empty_like(o)
-        h3.route(p, qd, kd, ws, kv_sel=sel)
+        if routed:
+            h3.route(p, qd, kd, ws, kv_sel=sel)
         for _ in range(2):
             h3.forward_qk8(p, qd, kd, vd, seg_d, times_d, pen=pen, kv_sel=sel, ws=ws, qk8_ws=qws, out=o8)
         q0 = torch.cuda.Event(enable_timing=True)
@@ -472,6 +572,12 @@ def run_ours(args, rank, world, local_rank):
         qk8_rel = (num / den) ** 0.5
         del qws, o8
 
+    # the other measured configurations of the call, on this GPU (one process): the dense biased call at the
+    # full packing (the 60 % target's S, 391.7 TFLOP) and the mid clip's sparsity sweep
+    extra = None
+    if not args.no_extra and world == 1 and args.heads is None and args.workload == "full_combined":
+        extra = extra_configs(args, h3, dev, stream, host, qd, kd, vd, o)
+
     # max over ranks; with head sharding the job's work is the sum of the ranks' shares
     ms, e2e_ms, fwd_ms, route_ms, merge_ms, tail_ms, qk8_ms, quant_ms = max_over_ranks(
         [ms, e2e_ms, fwd_ms, route_ms, merge_ms, tail_ms, qk8_ms, quant_ms], world, dev)
@@ -490,13 +596,15 @@ def run_ours(args, rank, world, local_rank):
     attn_tflops = (local_flops if sharded else eff_flops) / (fwd_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
     route_bytes = 2 * H * p.n_video_blocks * 64 * d * 2  # Q and K video rows, read once by the pool
+    dense_run = args.workload == "full_dense"
     line = {
-        "metric": "effective attention TFLOP/s (S=116883, H=56, d=128, sparsity 0.90, penalty on)",
+        "metric": METRIC_DENSE if dense_run else METRIC,
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "strong" if sharded else "weak",
         "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded counter-based generator, cluster-mean Q/K)",
-        "config": {"workload": WORKLOAD, "H": cfg.H, "S": S, "d": d, "block": 64, "sparsity": sparsity,
+        "config": {"workload": WORKLOAD_DENSE if dense_run else WORKLOAD, "H": cfg.H, "S": S, "d": d, "block": 64,
+                   "sparsity": sparsity,
                    "parallelism": (f"head-sharded over {world} GPUs (rank 0: heads {h0}..{h0 + H - 1})" if sharded
                                    else f"{world} independent calls, one per GPU"),
                    "k": int(p.k), "seed": seed, "l2": "no flush: Q+K+V = 5.0 GB per step, far above the 126 MB L2",
@@ -508,8 +616,9 @@ def run_ours(args, rank, world, local_rank):
                      "kernel": "attn_kernel (fused routed attention); achieved = effective FLOPs per launch / "
                                "CUDA-event time of the forward call (kv_desc prep + attention)",
                      "peak_source": f"{peak_kind} bf16_tflops_sustained"},
-        "routing": {"ms": route_ms, "bytes_read": route_bytes, "gbs": route_bytes / (route_ms * 1e-3) / 1e9,
-                    "hbm_peak_gbs": peaks["hbm_gbs"]},
+        "routing": None if not routed else {
+            "ms": route_ms, "bytes_read": route_bytes, "gbs": route_bytes / (route_ms * 1e-3) / 1e9,
+            "hbm_peak_gbs": peaks["hbm_gbs"]},
         "merge": None if args.no_merge else {
             "kernel": "merge_kernel (h3attn_merge: two partitions, O bf16 [H][S][d] + LSE f32, out O + LSE)",
             "ms": merge_ms, "bytes": 3 * H * S * (d * 2 + 4),
@@ -525,7 +634,9 @@ def run_ours(args, rank, world, local_rank):
             "vs_bf16_forward": fwd_ms / qk8_ms,
             "quantize_gbs": (2 * H * S * d * 3 + 2 * H * p.n_blocks * 64 * 4) / (quant_ms * 1e-3) / 1e9,
             "rel_fro_vs_bf16": qk8_rel},
-        "gpu_launches": 6 * args.steps,  # pool_split, score_gemm, topk, kv_desc, pair, attn
+        "full_dense": None if extra is None else extra["full_dense"],
+        "mid_clip_sweep": None if extra is None else extra["mid_clip_sweep"],
+        "gpu_launches": (6 if routed else 2) * args.steps,  # pool_split, score_gemm, topk, kv_desc, pair, attn
         "clocks": clk,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms / args.steps},
@@ -533,7 +644,8 @@ def run_ours(args, rank, world, local_rank):
     if args.no_e2e:
         line["e2e"] = None
     if args.heads is not None:
-        line["config"]["workload"] = WORKLOAD.replace("H=56", f"H={args.heads}") + " (profiling variant)"
+        line["config"]["workload"] = line["config"]["workload"].replace("H=56", f"H={args.heads}") + \
+            " (profiling variant)"
     if not args.no_cpu_baseline and world == 1:
         small = inputs.custom(1, d, cfg.segments, seed, cluster_norm=cfg.cluster_norm)
         qs, ks, vs = (inputs.tensor(small, i) for i in range(3))
@@ -558,6 +670,11 @@ def main():
     ap.add_argument("--no-merge", action="store_true", help="skip the partition-merge measurement")
     ap.add_argument("--no-tail", action="store_true", help="skip the pooled-tail-term measurement")
     ap.add_argument("--no-qk8", action="store_true", help="skip the int8-QK measurement")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the dense full-size call and the mid-clip sparsity sweep (extra JSON keys)")
+    ap.add_argument("--workload", choices=["full_combined", "full_dense"], default="full_combined",
+                    help="the timed call: the routed headline workload (default) or the dense biased call at the "
+                         "same packing (profiling)")
     ap.add_argument("--shard", choices=["none", "heads"], default="none",
                     help="N>1: 'none' = one independent call per GPU (weak scaling); 'heads' = one call, its heads "
                          "split over the GPUs (strong scaling)")

@@ -26,7 +26,7 @@ SEG_TEXT, SEG_IMAGE_REF, SEG_AUDIO, SEG_GUIDE, SEG_OUTPUT = 0, 1, 2, 3, 4
 EXPORTS = ("h3attn_plan_init", "h3attn_workspace_bytes", "h3attn_pool", "h3attn_route", "h3attn_route_static",
            "h3attn_route_static_check",
            "h3attn_forward",
-           "h3attn_dense_workspace_bytes", "h3attn_dense_biased", "h3attn_check", "h3attn_selftest_timeout",
+           "h3attn_dense_workspace_bytes", "h3attn_dense_biased", "h3attn_check", "h3attn_selftest_timeout", "h3attn_set_wait_polls",
            "h3attn_attend_host", "h3attn_merge", "h3attn_tail_workspace_bytes", "h3attn_tail_correct",
            "h3attn_qk8_workspace_bytes", "h3attn_quantize_qk", "h3attn_forward_qk8",
            "h3attn_strerror")
@@ -109,6 +109,8 @@ def lib():
         L.h3attn_forward_qk8.restype = ctypes.c_int
         L.h3attn_check.argtypes = [_P, _P]
         L.h3attn_check.restype = ctypes.c_int
+        L.h3attn_set_wait_polls.argtypes = [ctypes.c_uint32]
+        L.h3attn_set_wait_polls.restype = ctypes.c_int
         L.h3attn_selftest_timeout.argtypes = [_P, ctypes.c_uint32, _P]
         L.h3attn_selftest_timeout.restype = ctypes.c_int
         L.h3attn_strerror.argtypes = [ctypes.c_int]
@@ -346,6 +348,12 @@ def tail_correct(p: Plan, v, kv_sel, o, lse, ws, tail_ws=None, stream=None) -> N
 def check(ws: torch.Tensor, stream=None) -> int:
     """Synchronise and return (and clear) the device status word."""
     return int(lib().h3attn_check(ws.data_ptr(), _stream(stream)))
+
+
+def set_wait_polls(polls: int) -> None:
+    """Test and diagnostics only: bound the attention kernels' waits of later calls to `polls` polls
+    (0 = default, no poll bound)."""
+    _raise(lib().h3attn_set_wait_polls(polls), "set_wait_polls")
 
 
 def selftest_timeout(ws: torch.Tensor, polls: int, stream=None) -> None:

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <atomic>
 #include <new>
 #include <cstdint>
 #include <cstring>
@@ -17,7 +18,10 @@ namespace {
 
 constexpr size_t kAlign = 256;
 constexpr size_t kStatusBytes = 256;
-constexpr uint32_t kWaitPolls = 0xFFFFFFFFu;
+constexpr uint32_t kWaitPolls = 0xFFFFFFFFu;  // no poll bound: only the time bound applies
+// poll bound of the attention kernels' waits for the calls launched next
+// (h3attn_set_wait_polls; 0 = kWaitPolls)
+std::atomic<uint32_t> g_wait_polls{0u};
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait: far above any legitimate stall
 using h3::kMaxSmem;
 
@@ -168,7 +172,8 @@ int forward_impl(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, 
     p.strength_log2 = pen->strength * log2e;
     p.cap_log2 = pen->cap * log2e;
   }
-  p.wait_polls = kWaitPolls;
+  const uint32_t polls = g_wait_polls.load(std::memory_order_relaxed);
+  p.wait_polls = polls == 0u ? kWaitPolls : polls;
   p.wait_ns = kWaitNs;
   // routed: adjacent pairs over the dense prefix, then the overlap pairing
   p.qpairs = routed ? reinterpret_cast<const uint32_t*>(wsb + wl.pairs) : nullptr;
@@ -534,6 +539,11 @@ int h3attn_check(void* ws, void* stream) {
   if (status == h3::kStatusTimeout) return H3ATTN_ETIMEOUT;
   if (status == h3::kStatusData) return H3ATTN_EDATA;
   return status == 0 ? H3ATTN_OK : H3ATTN_ECUDA;
+}
+
+int h3attn_set_wait_polls(uint32_t polls) {
+  g_wait_polls.store(polls, std::memory_order_relaxed);
+  return H3ATTN_OK;
 }
 
 int h3attn_selftest_timeout(void* ws, uint32_t polls, void* stream) {

@@ -631,6 +631,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       if (row_valid && part == 0 && p.lse != nullptr) p.lse[(size_t)head * p.S + qrow] = (m + __log2f(l)) * kLn2;
     }
+    // a step left early on a give-up may still have TMEM accesses in flight:
+    // they complete before the allocation is released
+    tmem_wait_st();
+    tmem_wait_ld();
   }
 
   tc_fence_before();

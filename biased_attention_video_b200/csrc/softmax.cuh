@@ -35,15 +35,17 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const A
   for (uint32_t i = 0;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
+    bool give_up = i >= p.wait_polls;
     if ((i & 1023u) == 1023u) {
       uint64_t now;
       asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
       if (t0 == 0) t0 = now;
-      if (i >= p.wait_polls || now - t0 > p.wait_ns) {
-        *abort = 1;
-        report(p.status, kStatusTimeout);
-        return false;
-      }
+      give_up = give_up || now - t0 > p.wait_ns;
+    }
+    if (give_up) {
+      *abort = 1;
+      report(p.status, kStatusTimeout);
+      return false;
     }
   }
 }

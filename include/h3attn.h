@@ -319,6 +319,18 @@ H3ATTN_API int h3attn_dense_biased(int H, int S, int d, const uint16_t* q, const
  * stream reports an error. */
 H3ATTN_API int h3attn_check(void* ws, void* stream);
 
+/* Test and diagnostics only: bound every device-side wait of the attention
+ * kernels launched by later calls (h3attn_forward, h3attn_dense_biased,
+ * h3attn_forward_qk8, h3attn_attend_host) to `polls` unsuccessful polls of its
+ * barrier; 0 restores the default (no poll bound).  The time bound of 2 s per
+ * wait always applies, and the waits that drain a give-up (for the kernel's
+ * own TMA loads and MMAs already in flight) are bounded by time only, so a
+ * kernel that gives up still lets its own copies complete before it exits.
+ * A wait that runs out records H3ATTN_ETIMEOUT in the workspace status word
+ * (h3attn_check reports and clears it) and the outputs of that call are not
+ * valid.  Process-wide; not synchronised with calls already launched. */
+H3ATTN_API int h3attn_set_wait_polls(uint32_t polls);
+
 /* Self-test of the bounded-wait mechanism: launches one block that waits on
  * an mbarrier nothing arrives at, with a limit of `polls` polls, and records
  * H3ATTN_ETIMEOUT in the status word when it gives up.  No other work. */

@@ -235,7 +235,7 @@ def test_routing_only_routed():
     _sampled_forward(cfg, 0.85, None, heads=list(range(8)), blocks=[0, 5, 9, 10, 11, 100, 200, 255])
 
 
-@pytest.mark.parametrize("sparsity", [0.0, 0.90])
+@pytest.mark.parametrize("sparsity", [0.0, 0.60, 0.85, 0.90])
 def test_mid_clip_sampled(sparsity):
     cfg = inputs.MID_CLIP
     _sampled_forward(cfg, sparsity, None, heads=[0, 31, 55], blocks=[0, 25, 26, 27, 28, 300, 600, 767])
@@ -247,6 +247,11 @@ def test_full_size_sampled(cfg):
     the guide/output boundary block 929, frame-straddling blocks and the 19-row tail."""
     _sampled_forward(cfg, cfg.sparsities[0], PEN, heads=[0, 55],
                      blocks=[0, 31, 32, 33, 34, 100, 500, 928, 929, 930, 1500, 1825, 1826])
+
+
+def test_full_combined_routing_all_heads():
+    """Workload 5 routing (S = 116,883, 1,794 video blocks, k = 180) for all 56 heads against the oracle."""
+    _route_and_compare(inputs.FULL_COMBINED, inputs.FULL_COMBINED.sparsities[0])
 
 
 # ---------------------------------------------------------- failure paths

@@ -53,6 +53,23 @@ def test_quantize_zero_and_scaled_rows():
     _check_quant(cfg, x)
 
 
+def test_quantize_rows_with_tiny_maximum():
+    """Rows whose max |x| is 2^-120 (finite 127 / max) and 2^-130 (a bf16 subnormal: 127 / max overflows in
+    fp32, so nonzero elements saturate to +-127 and zeros stay 0): the kernel takes the same fp32 decisions
+    as the oracle's quantiser (pinned by hand in the oracle pins)."""
+    cfg = inputs.custom(1, 128, _layout(10, 0, 1, 40, 1, 40), seed=63)
+    x = make(cfg, device=None)
+    q = x["q"].copy()
+    q[0, 2] = 0
+    q[0, 2, :4] = [0x0380, 0x0300, 0x8380, 0x0000]
+    q[0, 6] = 0
+    q[0, 6, :4] = [0x0008, 0x8004, 0x0000, 0x0001]
+    x["q"] = q
+    x["q_d"] = torch.from_numpy(q.view(np.int16)).cuda().view(torch.bfloat16)
+    x["k_d"] = torch.from_numpy(x["k"].view(np.int16)).cuda().view(torch.bfloat16)
+    _check_quant(cfg, x)
+
+
 def _qk8_all_rows(cfg, sparsity, pen, routed=True):
     x = make(cfg)
     p = h3.plan(cfg.H, cfg.S, cfg.d, x["seg"], sparsity=sparsity)

@@ -384,6 +384,26 @@ def test_tail_term_is_exact_for_blockwise_constant_inputs():
     assert np.abs(tail_o - dense_o).max() < 1e-12 and np.abs(tail_l - dense_l).max() < 1e-12
 
 
+def test_tail_term_weights_a_ragged_block_by_its_valid_rows():
+    """The last video block holds 32 valid rows (S = 608): with blockwise-constant inputs the dense result
+    counts that block's key 32 times, so the pooled term reproduces it only with the weight n_j = 32 (the
+    valid rows), not the block size 64."""
+    segs = [inputs.Segment(inputs.SEG_TEXT, 64), inputs.Segment(inputs.SEG_AUDIO, 64),
+            inputs.Segment(inputs.SEG_OUTPUT, 8 * 60, 8)]
+    cfg = inputs.custom(2, 32, segs, seed=13, cluster_norm=2.0)
+    seg, times, _ = cfg.layout()
+    assert cfg.S == 608 and cfg.S % 64 == 32
+    q, k, v = _blockwise_constant(cfg)
+    sel, _, _ = oracle.route(q, k, seg, 0.75)
+    last = cfg.S // 64
+    assert np.any(np.all(sel != last, axis=-1))                  # some query blocks drop the ragged block
+    H, S = 2, cfg.S
+    heads, rows = np.repeat(np.arange(H), S), np.tile(np.arange(S), H)
+    dense_o, dense_l = oracle.attend(q, k, v, seg, times, pen=None, sel=None, heads=heads, rows=rows)
+    tail_o, tail_l = oracle.attend_tail(q, k, v, seg, times, None, sel, heads, rows)
+    assert np.abs(tail_o - dense_o).max() < 1e-12 and np.abs(tail_l - dense_l).max() < 1e-12
+
+
 def test_tail_term_is_absent_without_dropped_blocks():
     segs = [inputs.Segment(inputs.SEG_TEXT, 64), inputs.Segment(inputs.SEG_OUTPUT, 4 * 64, 4)]
     cfg = inputs.custom(1, 32, segs, seed=4, cluster_norm=2.0)
@@ -412,6 +432,34 @@ def test_quantize_hand_row():
     codes, scales = oracle.quantize_rows(x)
     assert codes.tolist() == [[127, -64, 32, 16, 95, -127, 0, 64]]
     assert scales[0] == np.float32(1.0) / np.float32(127.0)
+
+
+def _f32_from_exact(num, den):
+    """The float32 nearest (ties to even) to (num / den) * 2^-149, for positive integers num, den with
+    num / den < 2^23 (the subnormal range, whose spacing is 2^-149)."""
+    from fractions import Fraction
+    v = Fraction(num, den)
+    n = v.numerator // v.denominator
+    r = v - n
+    if r > Fraction(1, 2) or (r == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    return np.array([n], np.uint32).view(np.float32)[0]
+
+
+def test_quantize_row_with_tiny_maximum():
+    """Rows whose max |x| is far below 1 (reading of the per-token rule: quotients and products in fp32).
+    Max 2^-120: 127/max = 127 * 2^120 is finite, so the codes are exact (half the max -> 63.5 -> 64).
+    Max 2^-130 (a bf16 subnormal): 127/max overflows to +inf in fp32, so every nonzero element takes the
+    code +-127 and zeros take 0 (0 * inf is NaN, read as 0).  The scales are max/127 rounded to fp32,
+    here subnormal: computed exactly by hand."""
+    x = np.zeros((2, 8), np.uint16)
+    x[0, :4] = [0x0380, 0x0300, 0x8380, 0x0000]   # 2^-120, 2^-121, -2^-120, 0
+    x[1, :4] = [0x0008, 0x8004, 0x0000, 0x0001]   # 2^-130, -2^-131, 0, 2^-133 (subnormal bf16)
+    codes, scales = oracle.quantize_rows(x)
+    assert codes[0].tolist() == [127, 64, -127, 0, 0, 0, 0, 0]
+    assert codes[1].tolist() == [127, -127, 0, 127, 0, 0, 0, 0]
+    assert scales[0] == _f32_from_exact(2 ** 29, 127)          # 2^-120 / 127 = 2^29 / 127 * 2^-149
+    assert scales[1] == _f32_from_exact(2 ** 19, 127)          # 2^-130 / 127
 
 
 def test_quantize_zero_row_and_power_of_two_invariance():
