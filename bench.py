@@ -44,7 +44,7 @@ METRIC_DENSE = "effective attention TFLOP/s (S=116883, H=56, d=128, dense, penal
 # 8-head launch of this packing, captured with --clock-control none), scaled by heads: a stored figure, not a
 # per-run measurement.  Valid only for the kernel sources it was taken from (attn.cu and softmax.cuh, hashed
 # together); reported as null once either changes.
-ATTN_TRAFFIC = {"source_sha256_prefix": "625bc0b48a1fbb0b", "bytes_per_head": (1.441045e9 + 0.231585e9) / 8}
+ATTN_TRAFFIC = {"source_sha256_prefix": "0c0252e010356b70", "bytes_per_head": (1.450940416e9 + 0.230045440e9) / 8}
 ATTN_SOURCES = ("attn.cu", "softmax.cuh")
 
 
@@ -358,11 +358,12 @@ def extra_configs(args, h3, dev, stream, host, qd, kd, vd, o):
         ms_call = _time_calls(torch, call, steps, warmup, stream)
         ms_fwd = _time_calls(torch, lambda: h3.forward(p, q3, k3, v3, seg_d, times_d, pen=None, kv_sel=sel, ws=ws,
                                                        out=o3), steps, 1, stream)
+        ms_route = _time_calls(torch, lambda: h3.route(p, q3, k3, ws, kv_sel=sel), steps, 1, stream) if routed else 0.0
         if h3.check(ws) != h3.OK:
             raise RuntimeError(f"device status after the mid-clip call at sparsity {s}")
         flops = 4.0 * cfg.d * effective_pairs(p, sel.cpu().numpy() if routed else None)
         sweep.append({"sparsity": s, "k": int(p.k), "ms_per_call": ms_call, "attention_ms": ms_fwd,
-                      "route_ms": ms_call - ms_fwd if routed else 0.0,
+                      "route_ms": ms_route,
                       "effective_tflop_per_call": flops / 1e12, "effective_tflops": flops / (ms_call * 1e-3) / 1e12,
                       "attention_tflops": flops / (ms_fwd * 1e-3) / 1e12,
                       "attention_frac_of_sustained_peak": flops / (ms_fwd * 1e-3) / 1e12 / peak})
