@@ -106,8 +106,10 @@ cudaError_t launch_pool(const uint16_t* x0, float* out0, const uint16_t* x1, flo
 bool encode_bf16_3d(CUtensorMap* map, const void* base, uint64_t dim0, uint64_t dim1, uint64_t dim2, uint32_t box0,
                     uint32_t box1);
 
-// Routing scratch (byte offsets): two-part bf16 pooled centroids of Q and K
-// [H][n_video][3 d] and the fp32 score matrix [H][n_video][ldc].
+// Routing scratch (byte offsets): the pooled centroids of Q and K as three
+// bf16 parts, [H][n_video][kSplitParts d], and the fp32 score matrix
+// [H][n_video][ldc].
+constexpr int kSplitParts = 6;
 struct RouteScratch {
   size_t qs, ks, scores, ldc, total;
 };

@@ -4,13 +4,15 @@
 //
 // Three kernels:
 //  1. pool_split_kernel: mean of every video block of Q and K (fp32 sums of the
-//     bf16 rows), written as two bf16 parts x = hi + lo (hi = bf16(x),
-//     lo = bf16(x - hi)), rows [hi | hi | lo] for Q and [hi | lo | hi] for K.
+//     bf16 rows), written as three bf16 parts x = h + m + l (h = bf16(x),
+//     m = bf16(x - h), l = bf16(x - h - m): together the 24 significant bits of
+//     the fp32 mean), rows [h | h | m | h | m | l] for Q and [h | m | h | l | m | h]
+//     for K.
 //  2. score_gemm_kernel: per head, scores = Qs . Ks^T over the concatenated
-//     3d-long rows, i.e. Qh.Kh + Qh.Kl + Ql.Kh -- the fp32 products of the
-//     pooled centroids up to the dropped Ql.Kl term and the residual of the
-//     two-part split (relative 2^-16 per product), on the tensor cores
-//     (tcgen05.mma kind::f16, fp32 accumulation in TMEM).
+//     6d-long rows, i.e. Qh.Kh + Qh.Km + Qm.Kh + Qh.Kl + Qm.Km + Ql.Kh -- every
+//     product of the pooled centroids' parts down to relative order 2^-16 (the
+//     dropped ones are below 2^-24), each exact in fp32, accumulated in fp32 on
+//     the tensor cores (tcgen05.mma kind::f16, fp32 accumulation in TMEM).
 //  3. topk_kernel: one warp per (head, query block): the k best key blocks,
 //     ties to the lower block, listed in ascending order.
 // The 1/sqrt(d) logit scale is a positive constant and does not change the
@@ -40,9 +42,10 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// One warp per (tensor, head, video block).  Output row layout (3d bf16):
-// Q: [hi | hi | lo], K: [hi | lo | hi] so that the row dot product of the two
-// concatenations is Qh.Kh + Qh.Kl + Ql.Kh.
+// One warp per (tensor, head, video block).  Output row layout (kSplitParts d
+// bf16): Q: [h | h | m | h | m | l], K: [h | m | h | l | m | h], so that the row
+// dot product of the two concatenations is Qh.Kh + Qh.Km + Qm.Kh + Qh.Kl +
+// Qm.Km + Ql.Kh.
 template <int D>
 __global__ void __launch_bounds__(256) pool_split_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
                                                          uint16_t* __restrict__ qs, uint16_t* __restrict__ ks, int H,
@@ -85,23 +88,27 @@ __global__ void __launch_bounds__(256) pool_split_kernel(const uint16_t* __restr
     for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xFFFFFFFFu, acc[i], o);
   if (rsub == 0) {
     const float inv = 1.0f / (float)nrows;
-    uint32_t hw[4], lw[4];
+    uint32_t hw[4], mw[4], lw[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
+      // the differences are exact in fp32: each part takes the next 8 significant bits
       const float a = acc[2 * i] * inv, b = acc[2 * i + 1] * inv;
       const float ah = __bfloat162float(__float2bfloat16_rn(a)), bh = __bfloat162float(__float2bfloat16_rn(b));
+      const float am = __bfloat162float(__float2bfloat16_rn(a - ah));
+      const float bm = __bfloat162float(__float2bfloat16_rn(b - bh));
       hw[i] = bf16x2_bits(ah, bh);
-      lw[i] = bf16x2_bits(a - ah, b - bh);
+      mw[i] = bf16x2_bits(am, bm);
+      lw[i] = bf16x2_bits((a - ah) - am, (b - bh) - bm);
     }
     const uint4 hv = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    const uint4 mv = make_uint4(mw[0], mw[1], mw[2], mw[3]);
     const uint4 lv = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-    uint16_t* dst_row = (t == 0 ? qs : ks) + ((size_t)h * n_video + vb) * (3 * D) + chunk * 8;
-    uint4* d0 = reinterpret_cast<uint4*>(dst_row);
-    uint4* d1 = reinterpret_cast<uint4*>(dst_row + D);
-    uint4* d2 = reinterpret_cast<uint4*>(dst_row + 2 * D);
-    *d0 = hv;
-    *d1 = t == 0 ? hv : lv;
-    *d2 = t == 0 ? lv : hv;
+    uint16_t* dst_row = (t == 0 ? qs : ks) + ((size_t)h * n_video + vb) * (kSplitParts * D) + chunk * 8;
+    const uint4 q_parts[kSplitParts] = {hv, hv, mv, hv, mv, lv};
+    const uint4 k_parts[kSplitParts] = {hv, mv, hv, lv, mv, hv};
+#pragma unroll
+    for (int part = 0; part < kSplitParts; ++part)
+      *reinterpret_cast<uint4*>(dst_row + part * D) = t == 0 ? q_parts[part] : k_parts[part];
   }
 }
 
@@ -571,7 +578,7 @@ __global__ void __launch_bounds__(256, 2) topk_reg_kernel(const float* __restric
 
 RouteScratch route_scratch_layout(int H, int d, int n_video) {
   RouteScratch r;
-  const size_t split = (size_t)H * n_video * 3 * d * sizeof(uint16_t);
+  const size_t split = (size_t)H * n_video * kSplitParts * d * sizeof(uint16_t);
   r.qs = 0;
   r.ks = (split + 255) / 256 * 256;
   r.scores = r.ks + (split + 255) / 256 * 256;
@@ -604,7 +611,8 @@ cudaError_t launch_route_pipeline(const uint16_t* q, const uint16_t* k, int32_t*
   if (e != cudaSuccess) return e;
   // 2. scores on the tensor cores
   CUtensorMap ta, tb;
-  if (!encode_bf16_3d(&ta, qs, 3 * d, n_video, H, 64, kGM) || !encode_bf16_3d(&tb, ks, 3 * d, n_video, H, 64, kGN))
+  if (!encode_bf16_3d(&ta, qs, kSplitParts * d, n_video, H, 64, kGM) ||
+      !encode_bf16_3d(&tb, ks, kSplitParts * d, n_video, H, 64, kGN))
     return cudaErrorInvalidValue;
   e = cudaFuncSetAttribute(score_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmem);
   if (e != cudaSuccess) return e;
@@ -618,7 +626,8 @@ cudaError_t launch_route_pipeline(const uint16_t* q, const uint16_t* k, int32_t*
   const int ggrid = (int)(tiles < n_sm ? tiles : n_sm);
   CUtensorMap tc;
   if (!encode_f32_3d(&tc, sc, n_video, n_video, H, r.ldc, 32, 32)) return cudaErrorInvalidValue;
-  score_gemm_kernel<<<ggrid, kGemmThreads, kGSmem, stream>>>(ta, tb, tc, n_video, 3 * d / 64, n_tm, n_tn, (int)tiles,
+  score_gemm_kernel<<<ggrid, kGemmThreads, kGSmem, stream>>>(ta, tb, tc, n_video, kSplitParts * d / 64, n_tm, n_tn,
+                                                             (int)tiles,
                                                              status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

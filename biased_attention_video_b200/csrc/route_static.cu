@@ -23,9 +23,9 @@
 
 namespace {
 
-// 32 MiB: a 256-byte status header, then the routing scratch (two-part pooled
-// centroids and the score matrix).
-constexpr size_t kStaticBytes = size_t(32) << 20;
+// 64 MiB: a 256-byte status header, then the routing scratch (the three-part
+// bf16 pooled centroids and the score matrix).
+constexpr size_t kStaticBytes = size_t(64) << 20;
 constexpr size_t kStatusHeader = 256;
 constexpr int kMaxDevices = 64;
 

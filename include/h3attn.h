@@ -122,9 +122,9 @@ H3ATTN_API int h3attn_plan_init(h3attn_plan* plan, int H, int S, int d, int bloc
  * guide times and a bitmap of the key blocks that need per-key handling,
  * about 0.5 MB at S = 116,883; the query-block pair table of a routed
  * forward, 4 bytes per head and 128-row tile of video query blocks, about
- * 0.2 MB at S = 116,883, H = 56; and the routing scratch: two-part bf16 pooled
- * Q and K of the video blocks and the fp32 pooled-score matrix, about 0.9 GB
- * at S = 116,883, H = 56, d = 128).
+ * 0.2 MB at S = 116,883, H = 56; and the routing scratch: three-part bf16
+ * pooled Q and K of the video blocks, six d-long parts per row, and the fp32
+ * pooled-score matrix, about 1.2 GB at S = 116,883, H = 56, d = 128).
  * The caller allocates it once, zero-filled (the first 256 bytes hold the
  * status word that h3attn_check reads and clears). */
 H3ATTN_API size_t h3attn_workspace_bytes(const h3attn_plan* plan);
@@ -142,9 +142,10 @@ H3ATTN_API int h3attn_pool(const h3attn_plan* plan, const uint16_t* x, int first
  *   kv_sel[h][i][0..k) = the k video key blocks j with the highest
  *   Qp[h][i].Kp[h][j] / sqrt(d), ties to the lower block, listed as absolute
  *   block indices in ascending order.  Qp, Kp are fp32 block means; the dot
- *   products run on the tensor cores over two-part bf16 splits of them
- *   (x = hi + lo, Qh.Kh + Qh.Kl + Ql.Kh accumulated in fp32: relative error
- *   about 2^-16 per product).
+ *   products run on the tensor cores over three-part bf16 splits of them
+ *   (x = h + m + l, the 24 significant bits of the fp32 mean; the six
+ *   products of parts down to relative order 2^-16, each exact, accumulated
+ *   in fp32: the dropped ones are below 2^-24 of the product).
  * q, k: bf16 [H][S][d] device; kv_sel: int32 [H][n_video_blocks][k] device.
  * ws: workspace of at least h3attn_workspace_bytes(plan) bytes. */
 H3ATTN_API int h3attn_route(const h3attn_plan* plan, const uint16_t* q, const uint16_t* k, int32_t* kv_sel,
@@ -155,12 +156,12 @@ H3ATTN_API int h3attn_route(const h3attn_plan* plan, const uint16_t* q, const ui
  * device memory when they route (a framework that owns all device memory
  * through its own pool, a loop that must not pay cudaMalloc's implicit
  * synchronisation, a host with a fixed memory budget).
- * Same result as h3attn_route.  Its scratch (the two-part bf16 pooled
- * centroids of Q and K and the fp32 score matrix) is a fixed 32 MiB array
+ * Same result as h3attn_route.  Its scratch (the three-part bf16 pooled
+ * centroids of Q and K and the fp32 score matrix) is a fixed 64 MiB array
  * inside the library that every GPU loading the library holds until the
  * process exits; its first 256 bytes are the status word of these calls, and
- * problems needing more than the remaining 32 MiB - 256 bytes, i.e. with
- * 12 * H * n_video_blocks * d + 16 * H * n_video_blocks * ceil(n_video_blocks / 4)
+ * problems needing more than the remaining 64 MiB - 256 bytes, i.e. with
+ * 24 * H * n_video_blocks * d + 16 * H * n_video_blocks * ceil(n_video_blocks / 4)
  * bytes above that, are rejected with H3ATTN_EWORKSPACE.  Every call overwrites
  * all the scratch it reads, so nothing needs clearing between calls; calls
  * that overlap on the GPU (other streams, other threads) share the array and

@@ -86,6 +86,23 @@ def test_plan_rejects_bad_arguments():
     assert e.value.code == h3.EINVAL
 
 
+def test_plan_size_limits():
+    """The largest sequence is 8,192 blocks (S = 524,288: block ids fit the kernels' 14-bit list entries and the
+    lists fit shared memory); one row more, S = 0 or H = 0 is rejected before any device work."""
+    S = 8192 * 64
+    seg = np.concatenate([np.zeros(640, np.uint8), np.full(S - 640, 4, np.uint8)])
+    p = h3.plan(1, S, 128, seg, sparsity=0.9)
+    assert (p.n_blocks, p.first_video_block, p.n_video_blocks, p.k) == (8192, 10, 8182, 819)
+    seg1 = np.concatenate([seg, np.full(1, 4, np.uint8)])
+    with pytest.raises(h3.H3Error) as e:
+        h3.plan(1, S + 1, 128, seg1)
+    assert e.value.code == h3.EUNSUPPORTED
+    seg0 = np.zeros(128, np.uint8)
+    for H, SS in ((0, 128), (1, 0), (1, -5)):
+        out = h3.Plan()
+        assert h3.lib().h3attn_plan_init(ctypes.byref(out), H, SS, 128, 64, 0.0, seg0.ctypes.data) == h3.EINVAL
+
+
 def test_plan_without_video_is_dense():
     seg = np.zeros(300, np.uint8)
     p = h3.plan(1, 300, 64, seg)

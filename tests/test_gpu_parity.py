@@ -64,8 +64,8 @@ def test_route_routing_only():
 
 
 @pytest.mark.parametrize("sparsity", [0.0, 0.60, 0.85, 0.90])
-def test_route_mid_clip_sampled_heads(sparsity):
-    _route_and_compare(inputs.MID_CLIP, sparsity, heads=[0, 27, 55])
+def test_route_mid_clip_all_heads(sparsity):
+    _route_and_compare(inputs.MID_CLIP, sparsity)
 
 
 def test_route_more_than_2048_video_blocks():
@@ -247,6 +247,27 @@ def test_full_size_sampled(cfg):
     the guide/output boundary block 929, frame-straddling blocks and the 19-row tail."""
     _sampled_forward(cfg, cfg.sparsities[0], PEN, heads=[0, 55],
                      blocks=[0, 31, 32, 33, 34, 100, 500, 928, 929, 930, 1500, 1825, 1826])
+
+
+def test_maximum_sequence_length():
+    """The largest supported sequence, S = 524,288 (8,192 blocks; 8,182 video blocks routed to k = 819 at
+    sparsity 0.9 by the shared-memory top-k), one head, d = 128, guide and output video with the penalty: routing
+    of every video query block, then sampled rows of the prefix, the first video blocks, the guide/output boundary
+    and the last block against the oracle."""
+    segs = _layout(256, 384, 32, 8182, 32, 8182)
+    cfg = inputs.custom(1, 128, segs, seed=81, cluster_norm=2.0)
+    assert cfg.S == 524288
+    p, x, sel, ws = _route_and_compare(cfg, 0.9)
+    assert (p.n_blocks, p.n_video_blocks, p.k) == (8192, 8182, 819)
+    o, l = h3.forward(p, x["q_d"], x["k_d"], x["v_d"], x["seg_d"], x["times_d"], pen=PEN,
+                      kv_sel=torch.from_numpy(sel).cuda(), ws=ws, lse=True)
+    assert h3.check(ws) == h3.OK
+    boundary = (256 + 384 + 32 * 8182) // 64
+    rows = sample_rows(cfg.S, [0, 9, 10, 11, 4000, boundary, boundary + 1, 8190, 8191], rows_per_block=(0, 31, 63))
+    ref_o, ref_l = oracle.attend(x["q"], x["k"], x["v"], x["seg"], x["times"], pen=PEN, sel=sel,
+                                 heads=np.zeros(len(rows), np.int32), rows=rows)
+    compare_outputs(host_bits(o)[0, rows], ref_o, "S = 524,288")
+    assert np.abs(l.cpu().numpy()[0, rows] - ref_l).max() <= LSE_ABS
 
 
 def test_full_combined_routing_all_heads():
