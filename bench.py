@@ -44,7 +44,7 @@ METRIC_DENSE = "effective attention TFLOP/s (S=116883, H=56, d=128, dense, penal
 # 8-head launch of this packing, captured with --clock-control none), scaled by heads: a stored figure, not a
 # per-run measurement.  Valid only for the kernel sources it was taken from (attn.cu and softmax.cuh, hashed
 # together); reported as null once either changes.
-ATTN_TRAFFIC = {"source_sha256_prefix": "0c0252e010356b70", "bytes_per_head": (1.450940416e9 + 0.230045440e9) / 8}
+ATTN_TRAFFIC = {"source_sha256_prefix": "25f4d281eb729407", "bytes_per_head": (1.589049344e9 + 0.234848000e9) / 8}
 ATTN_SOURCES = ("attn.cu", "softmax.cuh")
 
 
@@ -88,17 +88,16 @@ def effective_pairs(p, sel: np.ndarray | None) -> int:
 
 def executed_mma_pairs(p, sel: np.ndarray | None) -> int:
     """(query, key) pairs the tensor cores actually process: per 128-row tile, the union
-    of its two query blocks' key lists, rounded up to 128-key tiles.  The tiles are the
+    of its two query blocks' key lists, one 64-key block per step.  The tiles are the
     kernel's: adjacent blocks over the dense prefix (rounded up to an even block), then
     the video blocks paired within groups of 32 by greedy largest list overlap (ties to
     the lowest pair), an odd block out alone."""
     nkb = p.n_blocks
-    full = (nkb + 1) // 2                     # 128-key tiles of a dense row block
     if sel is None:
-        return int(p.H) * full * 128 * full * 128
+        return int(p.H) * ((nkb + 1) // 2) * nkb * 128 * 64
     fvb, H, kk = p.first_video_block, int(p.H), sel.shape[2]
     n_dense = (fvb + 1) // 2
-    total = H * n_dense * full                # a dense block makes its tile dense
+    total = H * n_dense * nkb                 # a dense block makes its tile dense: every key block
     first = 2 * n_dense
     nv = nkb - fvb
     G = 32
@@ -118,12 +117,12 @@ def executed_mma_pairs(p, sel: np.ndarray | None) -> int:
             key = np.where(ok, ov * 1024 + tie[None, :], -1)
             c = key.argmax(axis=1)
             u = 2 * kk - ov[np.arange(H), c]
-            total += int(((u + fvb + 1) // 2).sum())
+            total += int((u + fvb).sum())
             alive[np.arange(H), iu[0][c]] = False
             alive[np.arange(H), iu[1][c]] = False
         if gs % 2:
-            total += H * ((kk + fvb + 1) // 2)
-    return int(total) * 128 * 128
+            total += H * (kk + fvb)
+    return int(total) * 128 * 64
 
 
 def rank_seed(base_seed: int, rank: int) -> int:

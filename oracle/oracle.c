@@ -15,8 +15,8 @@
  *  [SLA] "H3 SLA Attention" node page, "How it works" (pooled matmul, top
  *        1 - sparsity_ratio) and its inputs table (sparsity_ratio,
  *        block_size, protect_audio).
- *  [CFG] "Per-layer attention config LoRAs" (MiniMax-H3-Experiments
- *        docs/attention.md), "Experimental: audio/text protection"
+ *  [CFG] "Per-layer attention config LoRAs",
+ *        "Experimental: audio/text protection"
  *        (sink_keys "prefix", sink_queries "audio"; 64-token query blocks).
  *  [BRK] "H3 sparse-attention breakpoints: FL2VA, Ref2VA, and Turbo",
  *        "Results at a glance" (what "10 %" of video KV means).
