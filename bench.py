@@ -44,7 +44,7 @@ METRIC_DENSE = "effective attention TFLOP/s (S=116883, H=56, d=128, dense, penal
 # 8-head launch of this packing, captured with --clock-control none), scaled by heads: a stored figure, not a
 # per-run measurement.  Valid only for the kernel sources it was taken from (attn.cu and softmax.cuh, hashed
 # together); reported as null once either changes.
-ATTN_TRAFFIC = {"source_sha256_prefix": "25f4d281eb729407", "bytes_per_head": (1.508250624e9 + 0.232810240e9) / 8}
+ATTN_TRAFFIC = {"source_sha256_prefix": "c5dfca8afeb2c7de", "bytes_per_head": (1.843117568e9 + 0.230613760e9) / 8}
 ATTN_SOURCES = ("attn.cu", "softmax.cuh")
 
 

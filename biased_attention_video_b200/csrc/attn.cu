@@ -141,12 +141,20 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // Tile order: head-major, so the ~300 CTAs resident at a time share one or
-  // two heads' K/V in L2; inside a head the dense (prefix) query tiles come
-  // first, so the longest tiles start earliest.
-  const int n_qtiles = p.n_dense_tiles + p.n_paired_tiles;
-  const int head = (int)(blockIdx.x / n_qtiles);
-  const int qtile = (int)(blockIdx.x % n_qtiles);
+  // Tile order: the dense (prefix) query tiles of every head first -- they
+  // walk every key block, so the longest tiles start earliest and none is left
+  // running alone at the end -- then the paired tiles head-major, so the ~300
+  // CTAs resident at a time share one or two heads' K/V in L2.
+  const int n_dense_all = p.H * p.n_dense_tiles;
+  int head, qtile;
+  if ((int)blockIdx.x < n_dense_all) {
+    head = (int)blockIdx.x / p.n_dense_tiles;
+    qtile = (int)blockIdx.x % p.n_dense_tiles;
+  } else {
+    const int b = (int)blockIdx.x - n_dense_all;
+    head = b / p.n_paired_tiles;
+    qtile = p.n_dense_tiles + b % p.n_paired_tiles;
+  }
   // An earlier CTA that gave up leaves the status word set: skip the work
   // (decided once per CTA so that every thread leaves together).
   if (tid == 0) *abort_flag = *reinterpret_cast<volatile int*>(p.status) == kStatusTimeout ? 1 : 0;
