@@ -41,7 +41,7 @@ METRIC_DENSE = "effective attention TFLOP/s (S=116883, H=56, d=128, dense, penal
 
 
 # DRAM bytes of one attn_kernel launch as ncu counted them (dram__bytes_read.sum + dram__bytes_write.sum of one
-# 8-head launch of this packing, captured with --clock-control none), scaled by heads: a stored figure, not a
+# 8-head launch of the routed packing, captured with --clock-control none), scaled by heads: a stored figure, not a
 # per-run measurement.  Valid only for the kernel sources it was taken from (attn.cu and softmax.cuh, hashed
 # together); reported as null once either changes.
 ATTN_TRAFFIC = {"source_sha256_prefix": "c5dfca8afeb2c7de", "bytes_per_head": (1.843117568e9 + 0.230613760e9) / 8}
@@ -612,7 +612,9 @@ def run_ours(args, rank, world, local_rank):
                    "executed_mma_tflop_per_call": 4 * d * mma_pairs / 1e12,
                    "route_ms": route_ms, "attention_ms": fwd_ms},
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak, "unit": "TFLOP/s",
-                     "frac": attn_tflops / peak, "traffic": attn_traffic_bytes(H),
+                     "frac": attn_tflops / peak,
+                     # the stored capture is of the routed workload; the dense one has none
+                     "traffic": None if dense_run else attn_traffic_bytes(H),
                      "kernel": "attn_kernel (fused routed attention); achieved = effective FLOPs per launch / "
                                "CUDA-event time of the forward call (kv_desc prep + attention)",
                      "peak_source": f"{peak_kind} bf16_tflops_sustained"},

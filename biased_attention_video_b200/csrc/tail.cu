@@ -107,12 +107,15 @@ __global__ void __launch_bounds__(256) tail_weights_kernel(const float* __restri
     if ((kept[j >> 5] >> (j & 31)) & 1u) return -INFINITY;
     return fmaf(srow[j], scale, j == n_video - 1 ? log_last : log_full);
   };
+  // unrolled so that several score loads are in flight per lane
   float m = -INFINITY;
+#pragma unroll 8
   for (int j = lane; j < n_video; j += 32) m = fmaxf(m, logit(j));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
   uint16_t* wrow = w + (size_t)row * ldk;
   float sum = 0.0f;
+#pragma unroll 8
   for (int j = lane; j < ldk; j += 32) {
     uint16_t b = 0;
     if (j < n_video && m > -INFINITY) {
@@ -260,41 +263,59 @@ __global__ void __launch_bounds__(128) tail_gemm_kernel(const __grid_constant__ 
 
 // ------------------------------------------------------------------ 4. merge
 // D / 8 threads per row of a video query block, 16 bytes each: O and LSE of
-// the row merged in place with the block's tail partition.
+// the row merged in place with the block's tail partition.  Each thread takes
+// kMergeRows rows (a block's passes kRowsPerPass rows apart), loading all of
+// them before merging any, so that several 16-byte loads are in flight.
+constexpr int kMergeRows = 4;
+
 template <int D>
 __global__ void __launch_bounds__(256) tail_merge_kernel(uint16_t* __restrict__ o, float* __restrict__ lse,
                                                          const uint16_t* __restrict__ ot,
                                                          const float* __restrict__ lt, int H, int S,
                                                          int first_block, int n_video) {
   constexpr int kThreadsPerRow = D / 8;
-  constexpr int kRowsPerBlock = 256 / kThreadsPerRow;
+  constexpr int kRowsPerPass = 256 / kThreadsPerRow;
   const long long video_rows = (long long)S - (long long)first_block * kBlock;
-  const long long t = (long long)blockIdx.x * kRowsPerBlock + threadIdx.x / kThreadsPerRow;
-  if (t >= (long long)H * video_rows) return;
+  const long long total = (long long)H * video_rows;
+  const long long t0 = (long long)blockIdx.x * kRowsPerPass * kMergeRows + threadIdx.x / kThreadsPerRow;
   const int sub = threadIdx.x % kThreadsPerRow;
-  const int h = (int)(t / video_rows);
-  const long long r = (long long)first_block * kBlock + t % video_rows;  // sequence row
-  const int i = (int)(r / kBlock) - first_block;                         // its video query block
-  const long long orow = (long long)h * S + r;
-  uint4* op = reinterpret_cast<uint4*>(o + orow * D) + sub;
-  const uint4 a = *op;
-  const uint4 b = __ldg(reinterpret_cast<const uint4*>(ot + ((size_t)h * n_video + i) * D) + sub);
-  const float la = lse[orow], lb = __ldg(lt + (size_t)h * n_video + i);
-  const float m = fmaxf(la, lb);
-  if (m == -INFINITY) return;  // nothing on either side: leave the row as it is
-  const float L = m + __logf(__expf(la - m) + __expf(lb - m));
-  const float wa = __expf(la - L), wb = __expf(lb - L);
-  const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
-  uint32_t out[4];
+  uint4 a[kMergeRows], b[kMergeRows];
+  float la[kMergeRows], lb[kMergeRows];
+  long long orow[kMergeRows];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const float lo = fmaf(wa, __uint_as_float(aw[q] << 16), wb * __uint_as_float(bw[q] << 16));
-    const float hi = fmaf(wa, __uint_as_float(aw[q] & 0xFFFF0000u), wb * __uint_as_float(bw[q] & 0xFFFF0000u));
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    out[q] = *reinterpret_cast<uint32_t*>(&v);
+  for (int k = 0; k < kMergeRows; ++k) {
+    const long long t = t0 + (long long)k * kRowsPerPass;
+    orow[k] = -1;
+    if (t < total) {
+      const int h = (int)(t / video_rows);
+      const long long r = (long long)first_block * kBlock + t % video_rows;  // sequence row
+      const int i = (int)(r / kBlock) - first_block;                         // its video query block
+      orow[k] = (long long)h * S + r;
+      a[k] = *(reinterpret_cast<const uint4*>(o + orow[k] * D) + sub);
+      b[k] = __ldg(reinterpret_cast<const uint4*>(ot + ((size_t)h * n_video + i) * D) + sub);
+      la[k] = lse[orow[k]];
+      lb[k] = __ldg(lt + (size_t)h * n_video + i);
+    }
   }
-  *op = make_uint4(out[0], out[1], out[2], out[3]);
-  if (sub == 0) lse[orow] = L;
+#pragma unroll
+  for (int k = 0; k < kMergeRows; ++k) {
+    if (orow[k] < 0) continue;
+    const float m = fmaxf(la[k], lb[k]);
+    if (m == -INFINITY) continue;  // nothing on either side: leave the row as it is
+    const float L = m + __logf(__expf(la[k] - m) + __expf(lb[k] - m));
+    const float wa = __expf(la[k] - L), wb = __expf(lb[k] - L);
+    const uint32_t aw[4] = {a[k].x, a[k].y, a[k].z, a[k].w}, bw[4] = {b[k].x, b[k].y, b[k].z, b[k].w};
+    uint32_t out[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float lo = fmaf(wa, __uint_as_float(aw[q] << 16), wb * __uint_as_float(bw[q] << 16));
+      const float hi = fmaf(wa, __uint_as_float(aw[q] & 0xFFFF0000u), wb * __uint_as_float(bw[q] & 0xFFFF0000u));
+      __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+      out[q] = *reinterpret_cast<uint32_t*>(&v);
+    }
+    *(reinterpret_cast<uint4*>(o + orow[k] * D) + sub) = make_uint4(out[0], out[1], out[2], out[3]);
+    if (sub == 0) lse[orow[k]] = L;
+  }
 }
 
 }  // namespace
@@ -364,7 +385,7 @@ cudaError_t launch_tail(const uint16_t* v, const float* scores, size_t ldc, cons
   if (e != cudaSuccess) return e;
   // 4. merge into O / LSE
   const long long mrows = (long long)H * ((long long)S - (long long)first_block * kBlock);
-  const int rows_per_block = 256 / (d / 8);
+  const int rows_per_block = 256 / (d / 8) * kMergeRows;
   const unsigned mgrid = (unsigned)((mrows + rows_per_block - 1) / rows_per_block);
   if (mgrid > 0) {
     if (d == 64)
