@@ -57,3 +57,40 @@ def test_reference_arm_prints_one_line_with_the_contract_keys():
     with contextlib.redirect_stdout(out2):
         bench.run_reference(args, 1, 2)
     assert out2.getvalue() == ""
+
+
+class _Plan:
+    """The three plan fields the executed-work count reads."""
+
+    def __init__(self, H, n_blocks, first_video_block):
+        self.H, self.n_blocks, self.first_video_block = H, n_blocks, first_video_block
+
+
+def test_executed_work_of_a_dense_plan():
+    """Every 128-row tile walks every 64-key block."""
+    p = _Plan(3, 37, 0)
+    assert bench.executed_mma_pairs(p, None) == 3 * 19 * 37 * 128 * 64
+
+
+@pytest.mark.parametrize("fvb", [0, 3, 4])
+def test_executed_work_when_every_list_is_the_same(fvb):
+    """Identical routed lists: every pair's union is the list itself, so a paired tile walks the k routed blocks
+    plus the forced ones; the dense prefix tiles (adjacent pairs up to an even block) walk every block."""
+    H, nb, k = 2, 90, 7
+    nv = nb - fvb
+    rng = np.random.default_rng(5)
+    lst = np.sort(rng.choice(nv, k, replace=False)) + fvb
+    sel = np.broadcast_to(lst, (H, nv, k)).astype(np.int32)
+    n_dense = (fvb + 1) // 2
+    first = 2 * n_dense
+    n_paired_rows = nb - first
+    tiles = n_paired_rows // 2 + n_paired_rows % 2
+    expect = H * (n_dense * nb + tiles * (k + fvb)) * 128 * 64
+    assert bench.executed_mma_pairs(_Plan(H, nb, fvb), sel) == expect
+
+
+def test_executed_work_of_disjoint_pairs():
+    """Two video query blocks with disjoint lists: their tile walks both lists (2k blocks)."""
+    H, nb, k = 1, 2, 1
+    sel = np.array([[[0], [1]]], np.int32)
+    assert bench.executed_mma_pairs(_Plan(H, nb, 0), sel) == 2 * k * 128 * 64
