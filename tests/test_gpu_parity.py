@@ -179,6 +179,19 @@ def test_forward_routed_pairing_edges(segs, fvb, nb):
     assert p.first_video_block == fvb and p.n_blocks == nb
 
 
+@pytest.mark.parametrize("segs,sparsity,fvb,nb,k", [
+    (_layout(0, 0, 0, 0, 1, 192), 0.7, 0, 3, 1),       # all video, three blocks: a pair and a lone one-step tile
+    (_layout(0, 0, 2, 300, 2, 340), 0.999, 0, 20, 1),  # all video, k = 1: tiles of one or two steps
+    (_layout(100, 0, 0, 0, 1, 576), 0.95, 2, 11, 1),   # two forced blocks, k = 1
+])
+def test_forward_routed_single_block_lists(segs, sparsity, fvb, nb, k):
+    """Routed lists of one key block: the shortest tiles (a lone query block with one step, or a pair whose
+    union is one or two blocks), every row against the oracle."""
+    cfg = inputs.custom(2, 128, segs, seed=58, cluster_norm=2.0)
+    _, p = _forward_all_rows(cfg, sparsity, PEN, routed=True)
+    assert (p.first_video_block, p.n_blocks, p.k) == (fvb, nb, k)
+
+
 def test_tiny_dense_biased():
     cfg = inputs.TINY_DENSE
     x = make(cfg)
