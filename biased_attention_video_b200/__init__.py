@@ -193,7 +193,7 @@ def route(p: Plan, q: torch.Tensor, k: torch.Tensor, ws: torch.Tensor, kv_sel=No
 
 def route_static(p: Plan, q: torch.Tensor, k: torch.Tensor, kv_sel=None, stream=None) -> torch.Tensor:
     """Same result as route(), for callers that cannot allocate device memory: the
-    pooled centroids live in a fixed 32 MiB array inside the library (no workspace).
+    pooled centroids live in a fixed 64 MiB array inside the library (no workspace).
     The output buffer kv_sel may be passed in; concurrent calls share that array."""
     _check_qkv(q, k)
     if kv_sel is None:
